@@ -1,0 +1,479 @@
+"""Benchmark of the block-sparse prefill attention path on B200.
+
+One step = one pass of the whole path over one batch: pool (a1), block
+scores + routing (a2-a4) and exact + 0th-order attention (a5-a7).  Default
+workload: the DiT-video-shaped N = 32K case (B=1, H=12, d=128, top-k density
+0.15).  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--density X] [--impl psa|reference]
+
+Timing: W untimed warm-up steps, then K timed steps.  Each step is bracketed
+by CUDA events on the launching stream; a 512 MB buffer is rewritten between
+steps (outside the events) so L2 (126 MB) starts cold every step.  Multi-GPU
+(torchrun): every rank runs the same-size problem on its own seeded inputs
+(weak scaling, no collective on the data path); the step time is the max
+over ranks.  ``--impl reference`` times the fp64 CPU oracle on a bounded
+sample of the same workload (the only other place this file runs it).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_attention_psa_b200 import psa  # noqa: E402
+from block_sparse_attention_psa_b200.inputs import WORKLOADS, make_qkv  # noqa: E402
+
+METRIC = "block-sparse attn effective TFLOP/s & ms/call at N=32K; % of bf16 TC / HBM roofline"
+DEFAULT_WORKLOAD = "dit_video_n32k"
+L2_FLUSH_BYTES = 512 << 20
+
+
+# ---------------------------------------------------------------- accounting
+def dense_flops(B, H, N, d, causal):
+    """Dense-equivalent FLOPs of attention: 4 B H N^2 d (half when causal)."""
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def executed_flops(row_ptr, col_idx, B, H, M, d, causal):
+    """Algorithmic FLOPs the sparse path executes (host, from the block lists):
+    4 d b^2 per listed block pair (a causal diagonal block counts its b(b+1)/2
+    visible pairs) + 4 d b per 0th-order term (unlisted candidate)."""
+    b = 64
+    rp = row_ptr.astype(np.int64)
+    nsel = np.diff(rp)
+    rows = np.arange(B * H * M)
+    I = rows % M
+    if causal:
+        pcand = I                      # 0th-order candidates J < I
+        n_diag = len(rows)             # routers always list the diagonal
+        exact_pairs = b * b * (nsel.sum() - n_diag) + n_diag * b * (b + 1) // 2
+        unlisted = pcand - (nsel - 1)
+    else:
+        exact_pairs = b * b * nsel.sum()
+        unlisted = M - nsel
+    return 4.0 * d * exact_pairs + 4.0 * d * b * unlisted.sum()
+
+
+def pool_bytes(B, H, N, d):
+    M = N // 64
+    return 3 * B * H * N * d * 2 + 3 * B * H * M * d * 4
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.rows = []
+        self.proc = None
+        try:
+            self.target = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.target = None
+
+    def start(self):
+        cmd = ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if self.target:
+            cmd += ["--id=" + str(self.target)]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        smax = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in self.rows for n, val in zip(names, r[4:8]) if val.lower() == "active"})
+        power = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(self.rows),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------- GPU arm
+class Step:
+    """Device buffers and one step of the path for one workload."""
+
+    def __init__(self, name, density, seed, device):
+        w = dict(WORKLOADS[name])
+        self.name = name
+        self.w = w
+        self.B, self.H, self.N, self.d = w["B"], w["H"], w["N"], w["d"]
+        self.M = self.N // 64
+        self.causal = w["causal"]
+        self.keep_first = w["keep_first"]
+        self.mode, param = w["routing"]
+        if isinstance(param, tuple):
+            param = density if density is not None else param[0]
+        elif density is not None:
+            param = density
+        self.param = float(param)
+        q, k, v = make_qkv(self.B, self.H, self.N, self.d, w["gen"], seed)
+        self.host = [x.pin_memory() for x in (q, k, v)]
+        self.q, self.k, self.v = (x.to(device) for x in self.host)
+        B, H, M, d = self.B, self.H, self.M, self.d
+        f32 = dict(dtype=torch.float32, device=device)
+        self.stats = tuple(torch.empty(B, H, M, d, **f32) for _ in range(3))
+        cap = psa.psa_route_capacity(B, H, M, self.causal)
+        i32 = dict(dtype=torch.int32, device=device)
+        self.csr = (torch.empty(B * H * M + 1, **i32), torch.empty(cap, **i32), torch.empty(1, **i32))
+        self.ws = psa.workspace(B, H, self.N, d, device)
+        self.out = torch.empty_like(self.q)
+        self.out_host = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
+        self.stream = torch.cuda.current_stream()
+        # kernels of ours launched by one step
+        self.launches = 1 + (1 if self.mode == "topk" else 3) + 3
+
+    def run(self, ev=None):
+        """pool -> route -> attention; ``ev`` = 4 events to split the kernels."""
+        s = self.stream
+        if ev:
+            ev[0].record(s)
+        psa.psa_pool(self.q, self.k, self.v, out=self.stats, stream=s)
+        if ev:
+            ev[1].record(s)
+        qbar, kbar, vsum = self.stats
+        if self.mode == "topk":
+            psa.psa_route_topk(qbar, kbar, self.param, self.causal, out=self.csr, stream=s)
+        else:
+            psa.psa_route_thresh(qbar, kbar, self.param, self.causal, self.keep_first, ws=self.ws,
+                                 out=self.csr, stream=s)
+        if ev:
+            ev[2].record(s)
+        psa.psa_attn(self.q, self.k, self.v, kbar, vsum, self.csr[0], self.csr[1], self.causal, ws=self.ws,
+                     out=self.out, stream=s)
+        if ev:
+            ev[3].record(s)
+
+    def run_e2e(self):
+        """Host buffers in, host result out, through the same public calls."""
+        s = self.stream
+        for dst, src in zip((self.q, self.k, self.v), self.host):
+            dst.copy_(src, non_blocking=True)
+        self.run()
+        self.out_host.copy_(self.out, non_blocking=True)
+
+    def h2d_bytes(self):
+        return sum(x.numel() * x.element_size() for x in self.host)
+
+    def d2h_bytes(self):
+        return self.out_host.numel() * self.out_host.element_size()
+
+
+def _flush(buf):
+    buf.add_(1)
+
+
+def _dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def gpu_arm(args):
+    world, rank, local = _dist_setup()
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    device = torch.device("cuda", local)
+    st = Step(args.workload, args.density, seed=rank, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    for _ in range(args.warmup):
+        st.run()
+        _flush(flush)
+    torch.cuda.synchronize()
+
+    # routing of this batch, for the executed-FLOP count and density
+    rp = st.csr[0].cpu().numpy()
+    nnz = int(st.csr[2].item())
+    ci = st.csr[1][:nnz].cpu().numpy()
+    ex_flops = executed_flops(rp, ci, st.B, st.H, st.M, st.d, st.causal)
+    de_flops = dense_flops(st.B, st.H, st.N, st.d, st.causal)
+    n_cand = st.B * st.H * (st.M * (st.M + 1) // 2 if st.causal else st.M * st.M)
+    status = psa.psa_read_status(st.ws)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        st.run(evs[i])
+        _flush(flush)
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk = clocks.stop()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    pool_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    route_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    attn_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+
+    # end to end through the public API with host buffers
+    e2e_steps = max(1, min(args.steps, 5))
+    st.run_e2e()
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st.stream)
+    for _ in range(e2e_steps):
+        st.run_e2e()
+    e1.record(st.stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+
+    peaks = _peaks()
+    attn_avg = statistics.mean(attn_ms)
+    pool_avg = statistics.mean(pool_ms)
+    route_avg = statistics.mean(route_ms)
+    achieved = ex_flops / (attn_avg * 1e-3) / 1e12
+    tc_peak = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC,
+        "value": round(world * de_flops / (ms_per_step * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded generator, seed = rank)",
+        "config": {"workload": st.name, "B": st.B, "H": st.H, "N": st.N, "d": st.d, "block": 64,
+                   "causal": st.causal, "routing": f"{st.mode} {st.param}", "keep_first": st.keep_first,
+                   "parallelism": f"replicas x{world} (independent problems)" if world > 1 else "1 GPU",
+                   "l2": "flushed between steps (512 MB write outside the timed events)"},
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel (psa_attn call)",
+                     "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / tc_peak, 4), "traffic": None,
+                     "peak_source": peaks["source"] + " bf16 burst"},
+        "kernels": {"pool_ms": round(pool_avg, 4), "route_ms": round(route_avg, 4), "attn_ms": round(attn_avg, 4),
+                    "pool_gbs": round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3) / 1e9, 1),
+                    "pool_hbm_frac": round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3) / 1e9
+                                           / peaks["hbm_gbs"], 4),
+                    "attn_executed_tflops": round(achieved, 2),
+                    "attn_effective_tflops": round(de_flops / (attn_avg * 1e-3) / 1e12, 2)},
+        "flops": {"dense_equivalent": de_flops, "executed": ex_flops},
+        "density": {"realised": round(nnz / n_cand, 5), "listed_blocks": nnz},
+        "device_status": status,
+        "e2e": {"value": round(world * de_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": st.h2d_bytes(),
+                "d2h_bytes_per_step": st.d2h_bytes()},
+        "gpu_launches": st.launches * (args.steps),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(st.name, st.param, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- oracle arm
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("num_threads")]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_step_time(name, param, budget_s):
+    """Time the fp64 oracle on a bounded sample of one step of the workload:
+    pooling and block scores in full; routing of whole heads and attention on
+    a seeded sample of query blocks of those heads until the budget is spent;
+    both extrapolated (per head, per query block) to the whole step."""
+    import oracle.psa_oracle as O
+
+    w = WORKLOADS[name]
+    B, H, N, d = w["B"], w["H"], w["N"], w["d"]
+    M = N // 64
+    causal = w["causal"]
+    q, k, v = make_qkv(B, H, N, d, w["gen"], 0)
+    f64 = lambda t: t.double().numpy()
+    q, k, v = f64(q), f64(k), f64(v)
+    t0 = time.perf_counter()
+    qbar, kbar, vsum = O.pool(q, k, v)
+    s = O.block_scores(qbar, kbar)
+    t_full = time.perf_counter() - t0
+    mode = w["routing"][0]
+    rng = np.random.default_rng(0)
+    t_route, heads = 0.0, 0
+    t_attn, units = 0.0, 0
+    for bh in range(B * H):
+        b, h = divmod(bh, H)
+        t1 = time.perf_counter()
+        if mode == "topk":
+            rp, ci = O.route_topk(s[b:b + 1, h:h + 1], param, causal)
+        else:
+            rp, ci = O.route_thresh(s[b:b + 1, h:h + 1], param, causal, w["keep_first"])
+        t_route += time.perf_counter() - t1
+        heads += 1
+        for I in rng.permutation(M):
+            t1 = time.perf_counter()
+            O.attention(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1],
+                        kbar[b:b + 1, h:h + 1], vsum[b:b + 1, h:h + 1], rp, ci, causal, 64, [(0, 0, int(I))])
+            t_attn += time.perf_counter() - t1
+            units += 1
+            if t_route + t_attn > budget_s:
+                break
+        if t_route + t_attn > budget_s:
+            break
+    per_step = t_full + t_route / heads * (B * H) + t_attn / units * (B * H * M)
+    return per_step, units, B * H * M, t_full + t_route + t_attn
+
+
+def cpu_baseline(name, param, budget_s=15.0):
+    w = WORKLOADS[name]
+    per_step, done, total, spent = oracle_step_time(name, param, budget_s)
+    de = dense_flops(w["B"], w["H"], w["N"], w["d"], w["causal"])
+    return {"value": round(de / per_step / 1e12, 6), "unit": "TFLOP/s", "cores": _oracle_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 numpy oracle: pool + scores in full, routing + attention on {done} of {total} "
+                      f"query blocks ({spent:.1f} s), extrapolated per query block; {per_step:.1f} s/step",
+            "host_cpus": os.cpu_count()}
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    mode, param = w["routing"]
+    if isinstance(param, tuple):
+        param = param[0]
+    if args.density is not None:
+        param = args.density
+    budget = max(2.0, min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))
+    times = []
+    for i in range(args.warmup + args.steps):
+        per_step, done, total, spent = oracle_step_time(args.workload, param, budget)
+        if i >= args.warmup:
+            times.append(per_step)
+    ms = statistics.mean(times) * 1e3
+    de = dense_flops(w["B"], w["H"], w["N"], w["d"], w["causal"])
+    value = de / (ms * 1e-3) / 1e12
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator, seed 0)",
+        "config": {"workload": args.workload, "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
+                   "routing": f"{mode} {param}", "l2": "n/a (host)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _oracle_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: pool + scores in full, routing + attention on a sample of "
+                                   f"query blocks (~{budget:.0f} s), extrapolated per query block"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--density", type=float, default=None, help="override the routing parameter")
+    ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

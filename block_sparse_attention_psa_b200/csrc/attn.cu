@@ -1,0 +1,729 @@
+// attn.cu -- a5..a7: exact attention on the listed key blocks plus the
+// 0th-order term of every other candidate block, in one softmax.
+//
+// PISA summary (kodorricoding.tistory.com/108): routing table (listed blocks
+// exact with the original K/V tokens, the others through the block-mean key
+// and the value sum) and "Why approximating unselected blocks keeps softmax
+// intact" (both kinds of term in one accumulation, so the denominator stays
+// consistent).  FlashPrefill summary, 2.c "Index-driven physical jumping":
+// the K/V tiles are fetched straight from the block list, with no per-block
+// branch over masked blocks.
+//
+// Design (sm_100a):
+//  * One work unit = one query block (64 rows) of one head.  A block list
+//    belongs to a 64-row query block, so 128 query rows never share keys.
+//    To keep the tensor core at M = 128 the products are TRANSPOSED:
+//       S^T[128 keys x 64 queries]  = K_tile . Q^T     (A = 2 listed key
+//                                      blocks, K-major; B = Q, K-major)
+//       O^T[d x 64 queries]        += V_tile^T . P^T   (A = V, MN-major;
+//                                      B = P^T, MN-major)
+//    with S^T and O^T in TMEM (tcgen05.mma, f32 accumulate).
+//  * Softmax stabiliser: the per-query constant c_i = max_J (a_iJ + ln 64)
+//    over all candidate blocks, a_iJ = q_i.kbar_J/sqrt(d), taken in a first
+//    sweep over the pooled keys.  Because the mean of a block's logits is
+//    a_iJ, the largest term of the row is >= e^{c_i - ln 64}; every term
+//    relative to c_i stays in fp32 range unless one key's logit exceeds its
+//    block mean by ~90.  Rows whose final sum leaves [2^-60, 2^60] are
+//    recomputed exactly by a fixup kernel.  With a fixed stabiliser the
+//    running output never needs rescaling, so there is no correction step.
+//  * Tile stream of a unit: A1 tiles (pooled keys, for c), A2 tiles (pooled
+//    keys + pooled values of the unlisted blocks), E tiles (two listed key
+//    blocks each).  Warp 0: TMA producer.  Warp 1: tcgen05 issuer (one
+//    thread) and TMEM owner.  Warps 2-5: softmax + epilogue, one thread per
+//    TMEM lane (= key row of S^T, = feature row of O^T).
+//  * Every wait is bounded; on a timeout all roles stop, drain what is in
+//    flight, free TMEM and return with PSA_ERR_TIMEOUT recorded.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace psa {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;         // 128-byte column chunks
+  static constexpr int kQBytes = 64 * D * 2;     // one query block
+  static constexpr int kKVBytes = 128 * D * 2;   // two key blocks
+  static constexpr int kPBytes = 128 * 64 * 2;   // P^T tile
+  static constexpr int kOutBytes = 64 * D * 2;   // output staging
+  static constexpr int kNQ = 2, kNK = 2, kNV = 2, kNP = 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kNQ * kQBytes;
+  static constexpr int kOffV = kOffK + kNK * kKVBytes;
+  static constexpr int kOffP = kOffV + kNV * kKVBytes;
+  static constexpr int kOffOut = kOffP + kNP * kPBytes;
+  static constexpr int kOffMisc = kOffOut + kOutBytes;
+  // misc: 32 barriers (256 B) + tmem slot / flags (256 B) + red[4][64] +
+  // c2[64] + invl[64] + l[64] + bitmap[kMaxBlocks / 32]
+  static constexpr int kMiscBytes = 256 + 256 + 4 * 64 * 4 + 3 * 64 * 4 + kMaxBlocks / 8;
+  static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+  // kind::f16, bf16 x bf16 -> f32.  GEMM1: M=128 keys, N=64 queries, both
+  // K-major.  GEMM2: M=128 (feature rows), N=64 queries, both MN-major.
+  static constexpr uint32_t kIdesc1 = idesc_bf16_f32(128, 64, 0, 0);
+  static constexpr uint32_t kIdesc2 = idesc_bf16_f32(128, 64, 1, 1);
+};
+
+struct Params {
+  const int* row_ptr;
+  const int* col_idx;
+  long long col_cap;
+  __nv_bfloat16* out;
+  float* lse;
+  int BH, M, causal, dense, units;
+  float scale_log2;  // log2(e) / sqrt(d)
+  int* status;
+  int* fixup_count;
+  int* fixup_list;
+};
+
+// Everything every role needs to agree on about one work unit.
+struct Unit {
+  int bh, I, row, rp, nsel, cand, pcand, n_a1, n_a2, n_e, ntiles;
+  bool bad;  // row_ptr entries out of range
+};
+
+__device__ __forceinline__ Unit make_unit(int u, const Params& p) {
+  Unit x;
+  x.I = p.M - 1 - u / p.BH;  // largest I first (causal rows are the longest)
+  x.bh = u % p.BH;
+  x.row = x.bh * p.M + x.I;
+  x.cand = p.causal ? x.I + 1 : p.M;   // exact candidates J < cand
+  x.pcand = p.causal ? x.I : p.M;      // 0th-order candidates J < pcand
+  x.bad = false;
+  if (p.dense) {
+    x.rp = 0;
+    x.nsel = x.cand;
+  } else {
+    const int a = __ldg(p.row_ptr + x.row), b = __ldg(p.row_ptr + x.row + 1);
+    if (a < 0 || b < a || static_cast<long long>(b) > p.col_cap || b - a > x.cand) {
+      x.bad = true;
+      x.rp = 0;
+      x.nsel = 0;
+    } else {
+      x.rp = a;
+      x.nsel = b - a;
+    }
+  }
+  x.n_a1 = (x.cand + 127) / 128;
+  const bool a2 = !p.dense && x.pcand > 0 && x.nsel < x.cand;
+  x.n_a2 = a2 ? (x.pcand + 127) / 128 : 0;
+  int ne = (x.nsel + 1) / 2;
+  if (ne == 0 && x.n_a2 == 0) ne = 1;  // keep one product so O is defined
+  x.n_e = ne;
+  x.ntiles = x.n_a1 + x.n_a2 + x.n_e;
+  return x;
+}
+
+// tile t of a unit -> kind (0 = A1, 1 = A2, 2 = E) and index within the kind
+__device__ __forceinline__ void tile_kind(const Unit& x, int t, int& kind, int& ti) {
+  if (t < x.n_a1) {
+    kind = 0;
+    ti = t;
+  } else if (t < x.n_a1 + x.n_a2) {
+    kind = 1;
+    ti = t - x.n_a1;
+  } else {
+    kind = 2;
+    ti = t - x.n_a1 - x.n_a2;
+  }
+}
+
+// Bounded wait that ignores the abort flag (teardown only).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return;
+  }
+}
+
+// Column reduction over the 128 softmax threads: v[64] per thread,
+// out[q] = sum (or max) over threads of v[q].  Butterfly transpose-reduce
+// inside each warp (after it, lane L holds columns 2*rev5(L) and +1), then
+// the four warps combine through shared memory.
+template <bool kMax>
+__device__ __forceinline__ void group_reduce64(float (&v)[64], float* red, float* out, int lane, int wq,
+                                               int tid) {
+#pragma unroll
+  for (int step = 0; step < 5; ++step) {
+    const int o = 16 >> step;
+    const int half = 32 >> step;
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  const int col = ((lane & 16) ? 32 : 0) + ((lane & 8) ? 16 : 0) + ((lane & 4) ? 8 : 0) +
+                  ((lane & 2) ? 4 : 0) + ((lane & 1) ? 2 : 0);
+  red[wq * 64 + col] = v[0];
+  red[wq * 64 + col + 1] = v[1];
+  named_barrier_sync(1, 128);
+  if (tid < 64) {
+    const float a = red[tid], b = red[64 + tid], c = red[128 + tid], d = red[192 + tid];
+    out[tid] = kMax ? fmaxf(fmaxf(a, b), fmaxf(c, d)) : (a + b) + (c + d);
+  }
+  named_barrier_sync(1, 128);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
+                const __grid_constant__ CUtensorMap tmVb, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  uint8_t* sP = smem + C::kOffP;
+  uint8_t* sOut = smem + C::kOffOut;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffMisc);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 2;
+  uint64_t* k_full = bars + 4;
+  uint64_t* k_empty = bars + 6;
+  uint64_t* v_full = bars + 8;
+  uint64_t* v_empty = bars + 10;
+  uint64_t* s_full = bars + 12;
+  uint64_t* s_empty = bars + 14;
+  uint64_t* p_full = bars + 16;
+  uint64_t* p_empty = bars + 18;
+  uint64_t* o_full = bars + 20;
+  uint64_t* o_empty = bars + 22;
+  uint64_t* drain = bars + 24;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc + 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* unit_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile int* stop_s = reinterpret_cast<volatile int*>(tmem_slot + 3);
+  float* red = reinterpret_cast<float*>(smem + C::kOffMisc + 512);
+  float* c2s = red + 256;
+  float* invl = c2s + 64;
+  float* lsh = invl + 64;
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(lsh + 64);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&p_empty[i], 1);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *unit_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmKb);
+    tma_prefetch_desc(&tmVb);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int kc = 0, vc = 0, qc = 0;  // loads issued (lane 0's counts)
+    bool ok = true;
+    int ul = 0;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ul) {
+      const Unit x = make_unit(u, p);
+      const int qb = ul & 1;
+      if (lane == 0) {
+        ok = mbar_wait(&q_empty[qb], ((ul >> 1) & 1) ^ 1, abort_flag, p.status);
+        if (ok) {
+          mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(&tmQ, sQ + qb * C::kQBytes + c * 8192, &q_full[qb], 64 * c, 64 * x.I, x.bh);
+          ++qc;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      int colv = 0;
+      for (int t = 0; t < x.ntiles && ok; ++t) {
+        int kind, ti;
+        tile_kind(x, t, kind, ti);
+        int y0, y1;
+        const CUtensorMap* mk;
+        const CUtensorMap* mv;
+        if (kind == 2) {
+          mk = &tmK;
+          mv = &tmV;
+          const int e2 = 2 * ti;
+          int j1, j2;
+          if (p.dense) {
+            j1 = e2;
+            j2 = e2 + 1 < x.nsel ? e2 + 1 : e2;
+          } else {
+            if ((e2 & 31) == 0) {
+              const int idx = e2 + lane;
+              colv = (idx < x.nsel) ? __ldg(p.col_idx + x.rp + idx) : 0;
+            }
+            j1 = __shfl_sync(0xffffffffu, colv, e2 & 31);
+            j2 = __shfl_sync(0xffffffffu, colv, (e2 + 1) & 31);
+            if (e2 + 1 >= x.nsel) j2 = j1;
+          }
+          j1 = min(max(j1, 0), p.M - 1);
+          j2 = min(max(j2, 0), p.M - 1);
+          y0 = 64 * j1;
+          y1 = 64 * j2;
+        } else {
+          mk = &tmKb;
+          mv = &tmVb;
+          y0 = 128 * ti;
+          y1 = y0 + 64;
+        }
+        if (lane == 0) {
+          const int ks = kc % C::kNK;
+          ok = mbar_wait(&k_empty[ks], ((kc / C::kNK) & 1) ^ 1, abort_flag, p.status);
+          if (ok) {
+            mbar_arrive_expect_tx(&k_full[ks], C::kKVBytes);
+            uint8_t* dst = sK + ks * C::kKVBytes;
+#pragma unroll
+            for (int c = 0; c < C::kChunks; ++c) {
+              tma_load_3d(mk, dst + c * 16384, &k_full[ks], 64 * c, y0, x.bh);
+              tma_load_3d(mk, dst + c * 16384 + 8192, &k_full[ks], 64 * c, y1, x.bh);
+            }
+            ++kc;
+          }
+          if (ok && kind != 0) {
+            const int vs = vc % C::kNV;
+            ok = mbar_wait(&v_empty[vs], ((vc / C::kNV) & 1) ^ 1, abort_flag, p.status);
+            if (ok) {
+              mbar_arrive_expect_tx(&v_full[vs], C::kKVBytes);
+              uint8_t* dst = sV + vs * C::kKVBytes;
+#pragma unroll
+              for (int c = 0; c < C::kChunks; ++c) {
+                tma_load_3d(mv, dst + c * 16384, &v_full[vs], 64 * c, y0, x.bh);
+                tma_load_3d(mv, dst + c * 16384 + 8192, &v_full[vs], 64 * c, y1, x.bh);
+              }
+              ++vc;
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+    }
+    if (lane == 0) {
+      // make sure no bulk copy is still writing shared memory when we leave
+      for (int i = max(0, kc - C::kNK); i < kc; ++i) mbar_drain(&k_full[i % C::kNK], (i / C::kNK) & 1);
+      for (int i = max(0, vc - C::kNV); i < vc; ++i) mbar_drain(&v_full[i % C::kNV], (i / C::kNV) & 1);
+      for (int i = max(0, qc - C::kNQ); i < qc; ++i) mbar_drain(&q_full[i % C::kNQ], (i / C::kNQ) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int kc = 0, vc = 0, sc = 0, pc = 0;
+      bool ok = true;
+      bool pend = false, pend_first = false, pend_last = false;
+      int pend_ob = 0;
+      uint32_t pend_opar = 0;
+      auto issue_gemm2 = [&]() -> bool {
+        const int vs = vc % C::kNV, pb = pc & 1;
+        if (!mbar_wait(&v_full[vs], (vc / C::kNV) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(&p_full[pb], (pc >> 1) & 1, abort_flag, p.status)) return false;
+        if (pend_first && !mbar_wait(&o_empty[pend_ob], pend_opar, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t va = smem_u32(sV + vs * C::kKVBytes);
+        const uint32_t pa = smem_u32(sP + pb * C::kPBytes);
+        const uint32_t dt = tbase + 128 + 64 * pend_ob;
+        // A = V tile viewed MN-major (feature atoms 16 KB apart; for d = 64
+        // the second atom repeats the first and its rows are never read)
+        const uint32_t lbo = D == 128 ? 16384 : 0;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_bf16(dt, sdesc_sw128(va + kk * 2048, lbo, 1024), sdesc_sw128(pa + kk * 2048, 16, 1024),
+                      C::kIdesc2, (pend_first && kk == 0) ? 0u : 1u);
+        tc_commit(&v_empty[vs]);
+        tc_commit(&p_empty[pb]);
+        if (pend_last) tc_commit(&o_full[pend_ob]);
+        ++vc;
+        ++pc;
+        return true;
+      };
+      int ul = 0;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ul) {
+        const Unit x = make_unit(u, p);
+        const int qb = ul & 1;
+        if (!(ok = mbar_wait(&q_full[qb], (ul >> 1) & 1, abort_flag, p.status))) break;
+        const uint32_t qa = smem_u32(sQ + qb * C::kQBytes);
+        const int g2_total = x.n_a2 + x.n_e;
+        int g2_seen = 0;
+        for (int t = 0; t < x.ntiles; ++t) {
+          int kind, ti;
+          tile_kind(x, t, kind, ti);
+          const int ks = kc % C::kNK, sb = sc & 1;
+          if (!(ok = mbar_wait(&k_full[ks], (kc / C::kNK) & 1, abort_flag, p.status))) break;
+          if (!(ok = mbar_wait(&s_empty[sb], ((sc >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          const uint32_t ka = smem_u32(sK + ks * C::kKVBytes);
+          const uint32_t dt = tbase + 64 * sb;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            tc_mma_bf16(dt, sdesc_sw128(ka + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        sdesc_sw128(qa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), C::kIdesc1,
+                        kk > 0 ? 1u : 0u);
+          tc_commit(&k_empty[ks]);
+          tc_commit(&s_full[sb]);
+          if (t == x.ntiles - 1) tc_commit(&q_empty[qb]);
+          ++kc;
+          ++sc;
+          if (pend) {
+            pend = false;
+            if (!(ok = issue_gemm2())) break;
+          }
+          if (kind != 0) {
+            pend = true;
+            pend_ob = ul & 1;
+            pend_opar = ((ul >> 1) & 1) ^ 1;
+            pend_first = g2_seen == 0;
+            pend_last = g2_seen == g2_total - 1;
+            ++g2_seen;
+          }
+        }
+      }
+      if (ok && pend) ok = issue_gemm2();
+      // every MMA issued so far must finish before TMEM is freed
+      tc_commit(drain);
+      mbar_drain(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int wq = warp & 3;             // TMEM lane quarter of this warp
+    const int trow = wq * 32 + lane;     // TMEM lane: key row of S^T, feature row of O^T
+    const int tid = threadIdx.x - 64;    // 0..127 inside the group
+    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    float acc[64];   // running max in A1, then minus the stabiliser (log2 units)
+    float lsum[64];  // per-thread partial denominators
+    // Waits in this group never leave the control flow: after a timeout
+    // (abort raised) they return at once and the group runs on with garbage
+    // data until the next unit boundary, where all 128 threads take the same
+    // stop decision.  This keeps every named barrier matched.
+    int sc = 0, pc = 0;
+    int ul = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++ul) {
+      named_barrier_sync(1, 128);
+      if (tid == 0) *stop_s = *abort_flag;
+      named_barrier_sync(1, 128);
+      if (*stop_s) break;
+      const Unit x = make_unit(u, p);
+      if (!p.dense) {
+        // mark the listed blocks (A2 skips them) and validate the list
+        const int nw = (x.cand + 31) / 32;
+        for (int w = tid; w < nw; w += 128) bitmap[w] = 0u;
+        named_barrier_sync(1, 128);
+        bool bad = x.bad;
+        for (int i = tid; i < x.nsel; i += 128) {
+          const int J = __ldg(p.col_idx + x.rp + i);
+          if (J < 0 || J >= x.cand) {
+            bad = true;
+          } else {
+            const uint32_t bit = 1u << (J & 31);
+            if (atomicOr(&bitmap[J >> 5], bit) & bit) bad = true;
+          }
+        }
+        if (bad) record_status(p.status, kStatusCsr);
+        named_barrier_sync(1, 128);
+      }
+#pragma unroll
+      for (int q = 0; q < 64; ++q) {
+        acc[q] = -INFINITY;
+        lsum[q] = 0.f;
+      }
+      for (int t = 0; t < x.ntiles; ++t) {
+        int kind, ti;
+        tile_kind(x, t, kind, ti);
+        const int sb = sc & 1;
+        mbar_wait(&s_full[sb], (sc >> 1) & 1, abort_flag, p.status);
+        tc_fence_after();
+        const uint32_t sa = tbase + lane_addr + 64 * sb;
+        if (kind == 0) {
+          const bool valid = ti * 128 + trow < x.cand;
+          float sv[32];
+          tmem_ld32(sa, sv);
+          tc_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            if (valid) acc[q] = fmaxf(acc[q], sv[q]);
+          tmem_ld32(sa + 32, sv);
+          tc_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&s_empty[sb]);
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            if (valid) acc[32 + q] = fmaxf(acc[32 + q], sv[q]);
+          ++sc;
+          if (ti == x.n_a1 - 1) {
+            // stabiliser c2 = max_J a_iJ * log2(e) + log2(64)
+            group_reduce64<true>(acc, red, c2s, lane, wq, tid);
+            if (tid < 64) c2s[tid] = c2s[tid] * p.scale_log2 + 6.0f;
+            named_barrier_sync(1, 128);
+#pragma unroll
+            for (int q = 0; q < 64; ++q) acc[q] = -c2s[q];
+          }
+        } else {
+          bool valid, diag = false;
+          float add = 0.f;
+          if (kind == 1) {
+            const int J = ti * 128 + trow;
+            valid = J < x.pcand && !((bitmap[J >> 5] >> (J & 31)) & 1u);
+            add = 6.0f;  // weight 64 e^a on the value mean
+          } else {
+            const int idx = 2 * ti + (trow >> 6);
+            int J = -1;
+            if (idx < x.nsel) J = p.dense ? idx : __ldg(p.col_idx + x.rp + idx);
+            valid = J >= 0 && J < x.cand;
+            diag = p.causal && J == x.I;
+          }
+          const int kj = trow & 63;
+          const int pb = pc & 1;
+          uint8_t* prow = sP + pb * C::kPBytes + trow * 128;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float sv[32];
+            tmem_ld32(sa + 32 * h, sv);
+            tc_wait_ld();
+            if (h == 1) {
+              tc_fence_before();
+              mbar_arrive(&s_empty[sb]);
+            }
+            float pv[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const int qq = 32 * h + q;
+              float e = ex2_approx(fmaf(sv[q], p.scale_log2, acc[qq]) + add);
+              if (!valid || (diag && kj > qq)) e = 0.f;
+              lsum[qq] += e;
+              pv[q] = e;
+            }
+            if (h == 0) mbar_wait(&p_empty[pb], ((pc >> 1) & 1) ^ 1, abort_flag, p.status);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const int c = 4 * h + c4;
+              uint4 w;
+              w.x = pack_bf16x2(pv[8 * c4 + 0], pv[8 * c4 + 1]);
+              w.y = pack_bf16x2(pv[8 * c4 + 2], pv[8 * c4 + 3]);
+              w.z = pack_bf16x2(pv[8 * c4 + 4], pv[8 * c4 + 5]);
+              w.w = pack_bf16x2(pv[8 * c4 + 6], pv[8 * c4 + 7]);
+              *reinterpret_cast<uint4*>(prow + ((c ^ (trow & 7)) << 4)) = w;
+            }
+          }
+          fence_async_shared();
+          mbar_arrive(&p_full[pb]);
+          ++sc;
+          ++pc;
+        }
+      }
+
+      // ---------------------------------------------------------- epilogue
+      group_reduce64<false>(lsum, red, lsh, lane, wq, tid);
+      if (tid < 64) {
+        const float l = lsh[tid];
+        const bool good = l >= 0x1p-60f && l <= 0x1p60f;  // false for NaN
+        invl[tid] = good ? 1.0f / l : 0.f;
+        if (!good) *unit_flag = 1;
+        if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + tid] = (c2s[tid] + __log2f(l)) * kLn2;
+      }
+      if (tid == 0) bulk_wait_read0();  // the previous unit's store has read the staging tile
+      named_barrier_sync(1, 128);
+      const int ob = ul & 1;
+      mbar_wait(&o_full[ob], (ul >> 1) & 1, abort_flag, p.status);
+      tc_fence_after();
+      if (trow < D) {  // warp-uniform
+        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sOut);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float ov[32];
+          tmem_ld32(tbase + lane_addr + 128 + 64 * ob + 32 * h, ov);
+          tc_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            st[(32 * h + q) * D + trow] = __float2bfloat16_rn(ov[q] * invl[32 * h + q]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&o_empty[ob]);
+      fence_async_shared();
+      named_barrier_sync(1, 128);
+      if (tid == 0) {
+        bulk_store(p.out + static_cast<size_t>(x.row) * 64 * D, sOut, C::kOutBytes);
+        bulk_commit();
+        if (*unit_flag) {
+          const int slot = atomicAdd(p.fixup_count, 1);
+          p.fixup_list[slot] = u;
+          *unit_flag = 0;
+        }
+      }
+    }
+    if (tid == 0) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
+// ------------------------------------------------------------------ fixup
+// Exact two-pass recomputation (fp32, CUDA cores) of the units whose
+// denominator left the safe range under the fixed stabiliser.  One CTA of
+// 64 threads per listed unit, one thread per query row.  Rare path.
+template <int D>
+__global__ void __launch_bounds__(64) fixup_kernel(const __nv_bfloat16* __restrict__ q,
+                                                   const __nv_bfloat16* __restrict__ k,
+                                                   const __nv_bfloat16* __restrict__ v,
+                                                   const float* __restrict__ kbar, const float* __restrict__ vsum,
+                                                   Params p, int N) {
+  extern __shared__ float fx_sm[];
+  float(*qs)[D + 1] = reinterpret_cast<float(*)[D + 1]>(fx_sm);
+  float(*num)[D + 1] = reinterpret_cast<float(*)[D + 1]>(fx_sm + 64 * (D + 1));
+  uint32_t* listed = reinterpret_cast<uint32_t*>(fx_sm + 128 * (D + 1));
+  const int n = *p.fixup_count;
+  const int i = threadIdx.x;
+  const float tau = p.scale_log2 * kLn2;  // 1 / sqrt(d)
+  for (int f = blockIdx.x; f < n; f += gridDim.x) {
+    const Unit x = make_unit(p.fixup_list[f], p);
+    __syncthreads();
+    for (int w = i; w < (x.cand + 31) / 32; w += 64) listed[w] = 0u;
+    __syncthreads();
+    if (!p.dense) {
+      for (int e = i; e < x.nsel; e += 64) {
+        const int J = p.col_idx[x.rp + e];
+        if (J >= 0 && J < x.cand) atomicOr(&listed[J >> 5], 1u << (J & 31));
+      }
+    } else {
+      for (int J = i; J < x.cand; J += 64) atomicOr(&listed[J >> 5], 1u << (J & 31));
+    }
+    __syncthreads();
+    const size_t head = static_cast<size_t>(x.bh) * N;
+    const int qi = x.I * 64 + i;
+    for (int c = 0; c < D; ++c) {
+      qs[i][c] = __bfloat162float(q[(head + qi) * D + c]);
+      num[i][c] = 0.f;
+    }
+    float m = -INFINITY;
+    for (int pass = 0; pass < 2; ++pass) {
+      float den = 0.f;
+      for (int J = 0; J < x.cand; ++J) {
+        const bool on = (listed[J >> 5] >> (J & 31)) & 1u;
+        if (on) {
+          for (int j = 64 * J; j < 64 * J + 64; ++j) {
+            if (p.causal && j > qi) break;
+            float z = 0.f;
+            for (int c = 0; c < D; ++c) z = fmaf(qs[i][c], __bfloat162float(k[(head + j) * D + c]), z);
+            z *= tau;
+            if (pass == 0) {
+              m = fmaxf(m, z);
+            } else {
+              const float w = __expf(z - m);
+              den += w;
+              for (int c = 0; c < D; ++c) num[i][c] = fmaf(w, __bfloat162float(v[(head + j) * D + c]), num[i][c]);
+            }
+          }
+        } else if (J < x.pcand && kbar != nullptr) {
+          const size_t kb = (static_cast<size_t>(x.bh) * p.M + J) * D;
+          float a = 0.f;
+          for (int c = 0; c < D; ++c) a = fmaf(qs[i][c], kbar[kb + c], a);
+          a *= tau;
+          if (pass == 0) {
+            m = fmaxf(m, a + 4.1588830833596715f);  // + ln 64
+          } else {
+            const float w = __expf(a - m);
+            den += 64.f * w;
+            for (int c = 0; c < D; ++c) num[i][c] = fmaf(w, vsum[kb + c], num[i][c]);
+          }
+        }
+      }
+      if (pass == 1) {
+        const float r = 1.0f / den;
+        for (int c = 0; c < D; ++c) p.out[(head + qi) * D + c] = __float2bfloat16_rn(num[i][c] * r);
+        if (p.lse) p.lse[head + qi] = m + __logf(den);
+      }
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
+  using C = Cfg<D>;
+  CUtensorMap mq, mk, mv, mkb, mvb;
+  const uint64_t bh = static_cast<uint64_t>(a.BH);
+  if (encode_tensor_map_3d_bf16(&mq, a.q, D, a.N, bh, 64, 64) != CUDA_SUCCESS ||
+      encode_tensor_map_3d_bf16(&mk, a.k, D, a.N, bh, 64, 64) != CUDA_SUCCESS ||
+      encode_tensor_map_3d_bf16(&mv, a.v, D, a.N, bh, 64, 64) != CUDA_SUCCESS ||
+      encode_tensor_map_3d_bf16(&mkb, a.kbar_bf16, D, a.M, bh, 64, 64) != CUDA_SUCCESS ||
+      encode_tensor_map_3d_bf16(&mvb, a.dense ? a.kbar_bf16 : a.vbar_bf16, D, a.M, bh, 64, 64) !=
+          CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  Params p;
+  p.row_ptr = a.row_ptr;
+  p.col_idx = a.col_idx;
+  p.col_cap = a.col_cap;
+  p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.BH = a.BH;
+  p.M = a.M;
+  p.causal = a.causal;
+  p.dense = a.dense;
+  p.units = a.BH * a.M;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+  p.status = a.status;
+  p.fixup_count = a.fixup_count;
+  p.fixup_list = a.fixup_list;
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  const int grid = p.units < sms ? p.units : sms;
+  attn_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mkb, mvb, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t fx_smem = 128 * (D + 1) * sizeof(float) + kMaxBlocks / 8;
+  if ((e = cudaFuncSetAttribute(fixup_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(fx_smem))) != cudaSuccess)
+    return e;
+  fixup_kernel<D><<<64, 64, fx_smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(a.q),
+                                           reinterpret_cast<const __nv_bfloat16*>(a.k),
+                                           reinterpret_cast<const __nv_bfloat16*>(a.v), a.kbar32, a.vsum32, p,
+                                           a.N);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t st) {
+  return a.d == 128 ? launch_d<128>(a, st) : launch_d<64>(a, st);
+}
+
+}  // namespace psa

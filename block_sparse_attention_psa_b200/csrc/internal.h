@@ -1,0 +1,69 @@
+// internal.h -- launch helpers shared between the C-ABI layer (api.cu) and
+// the kernel files.  Not part of the public interface.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace psa {
+
+constexpr int kBlock = 64;        // tokens per block (the only supported size)
+constexpr int kMaxBlocks = 16384; // M limit (bitmaps and score rows on chip)
+
+// Workspace layout (byte offsets, each 256-aligned).  The header holds the
+// status word and the fixup counter.
+struct WorkspaceLayout {
+  size_t header = 0;        // int status; int fixup_count; ... (256 B)
+  size_t fixup_list = 0;    // int [B*H*M]
+  size_t kbar_bf16 = 0;     // bf16 [B*H*M*d]
+  size_t vbar_bf16 = 0;     // bf16 [B*H*M*d]
+  size_t row_count = 0;     // int [B*H*M]     (threshold routing)
+  size_t row_bits = 0;      // uint32 [B*H*M*ceil(M/32)]
+  size_t total = 0;
+};
+WorkspaceLayout workspace_layout(long long BH, long long M, long long d);
+
+// pool.cu
+cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int M, int d,
+                        float* qbar, float* kbar, float* vsum, cudaStream_t st);
+cudaError_t launch_pool_keys_bf16(const uint16_t* k, int BH, int M, int d, uint16_t* kbar_bf16,
+                                  cudaStream_t st);
+cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long n, uint16_t* kbar_bf16,
+                                 uint16_t* vbar_bf16, cudaStream_t st);
+
+// route.cu
+cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int M, int d, int k0, int causal,
+                              int* row_ptr, int* col_idx, long long total, int* nnz_out, cudaStream_t st);
+cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, int M, int d, float alpha,
+                                int causal, int keep_first, int* row_ptr, int* col_idx, long long capacity,
+                                int* nnz_out, int* row_count, uint32_t* row_bits, cudaStream_t st);
+
+// attn.cu
+struct AttnLaunch {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const uint16_t* kbar_bf16;
+  const uint16_t* vbar_bf16;
+  const float* kbar32;  // may be null in dense mode
+  const float* vsum32;  // may be null in dense mode
+  const int* row_ptr;   // null in dense mode
+  const int* col_idx;   // null in dense mode
+  long long col_cap;
+  uint16_t* out;
+  float* lse;
+  int BH, N, M, d, causal, dense;
+  int* status;
+  int* fixup_count;
+  int* fixup_list;
+};
+cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t st);
+
+// api.cu: driver entry point for cuTensorMapEncodeTiled (resolved once)
+CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                                   uint64_t outer, uint32_t box_inner, uint32_t box_rows);
+int device_sm_count();
+
+}  // namespace psa

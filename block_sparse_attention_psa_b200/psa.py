@@ -1,0 +1,223 @@
+"""Thin Python binding of the C ABI in ``include/psa.h`` (``libpsa.so``).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+Each function has the name of the C entry point it calls.  Tensors are
+PyTorch CUDA tensors (PyTorch is used for device memory and streams); the
+call is issued on ``torch.cuda.current_stream()`` unless a stream is given.
+A non-zero status raises :class:`PSAError`.  There is no fallback: if the
+library is missing, :func:`lib` raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpsa.so")
+
+PSA_OK = 0
+PSA_ERR_ARG = 1
+PSA_ERR_SHAPE = 2
+PSA_ERR_UNSUPPORTED = 3
+PSA_ERR_CAPACITY = 4
+PSA_ERR_CUDA = 5
+PSA_ERR_TIMEOUT = 6
+PSA_ERR_CSR = 7
+PSA_ERR_DEVICE = 8
+
+EXPORTS = ("psa_status_string", "psa_version", "psa_workspace_size", "psa_route_capacity", "psa_pool",
+           "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense", "psa_read_status")
+
+_lib = None
+
+
+class PSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: status {status}: {status_text(status)}")
+
+
+def _declare(L: ctypes.CDLL) -> None:
+    P, I, Z, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    sig = {
+        "psa_status_string": (ctypes.c_char_p, [I]),
+        "psa_version": (I, []),
+        "psa_workspace_size": (Z, [I, I, I, I]),
+        "psa_route_capacity": (Z, [I, I, I, I]),
+        "psa_pool": (I, [P, P, P, I, I, I, I, I, P, P, P, P]),
+        "psa_route_topk": (I, [P, P, I, I, I, I, F, I, P, P, Z, P, P]),
+        "psa_route_thresh": (I, [P, P, I, I, I, I, F, I, I, P, P, Z, P, P, Z, P]),
+        "psa_attn": (I, [P, P, P, P, P, P, P, Z, I, I, I, I, I, I, P, P, P, Z, P]),
+        "psa_dense": (I, [P, P, P, I, I, I, I, I, P, P, P, Z, P]),
+        "psa_read_status": (I, [P, ctypes.POINTER(I), P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m block_sparse_attention_psa_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        _declare(L)
+        _lib = L
+    return _lib
+
+
+def status_text(status: int) -> str:
+    return lib().psa_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != PSA_OK:
+        raise PSAError(fn, status)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _shape(q):
+    if q.dim() != 4 or q.dtype != torch.bfloat16:
+        raise ValueError("q, k, v must be bf16 [B, H, N, d]")
+    return tuple(int(x) for x in q.shape)
+
+
+def psa_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().psa_workspace_size(B, H, N, d))
+
+
+def psa_route_capacity(B: int, H: int, M: int, causal: bool) -> int:
+    return int(lib().psa_route_capacity(B, H, M, int(causal)))
+
+
+def workspace(B: int, H: int, N: int, d: int, device=None) -> torch.Tensor:
+    """A device workspace of psa_workspace_size bytes (256-byte aligned)."""
+    n = psa_workspace_size(B, H, N, d)
+    if n == 0:
+        raise PSAError("psa_workspace_size", PSA_ERR_ARG)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def psa_pool(q, k, v, block_size: int = 64, out=None, stream=None):
+    """Returns (qbar, kbar, vsum) float32 [B, H, M, d]."""
+    B, H, N, d = _shape(q)
+    M = N // block_size if block_size > 0 else 0
+    if out is None:
+        out = tuple(torch.empty(B, H, M, d, dtype=torch.float32, device=q.device) for _ in range(3))
+    qbar, kbar, vsum = out
+    _check("psa_pool", lib().psa_pool(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, block_size,
+                                      _ptr(qbar), _ptr(kbar), _ptr(vsum), _stream(stream)))
+    return qbar, kbar, vsum
+
+
+def psa_route_topk(qbar, kbar, density: float, causal: bool = False, capacity: int | None = None,
+                   out=None, stream=None):
+    """Returns (row_ptr, col_idx, nnz) device int32 tensors (nnz has one element)."""
+    B, H, M, d = (int(x) for x in qbar.shape)
+    if out is None:
+        cap = capacity if capacity is not None else psa_route_capacity(B, H, M, causal)
+        out = (torch.empty(B * H * M + 1, dtype=torch.int32, device=qbar.device),
+               torch.empty(max(cap, 1), dtype=torch.int32, device=qbar.device),
+               torch.empty(1, dtype=torch.int32, device=qbar.device))
+    row_ptr, col_idx, nnz = out
+    _check("psa_route_topk", lib().psa_route_topk(
+        _ptr(qbar), _ptr(kbar), B, H, M, d, float(density), int(causal), _ptr(row_ptr), _ptr(col_idx),
+        col_idx.numel(), _ptr(nnz), _stream(stream)))
+    return row_ptr, col_idx, nnz
+
+
+def psa_route_thresh(qbar, kbar, alpha: float, causal: bool = False, keep_first: bool = False,
+                     ws=None, capacity: int | None = None, out=None, stream=None):
+    """Returns (row_ptr, col_idx, nnz); nnz > col_idx.numel() means truncated."""
+    B, H, M, d = (int(x) for x in qbar.shape)
+    if ws is None:
+        ws = workspace(B, H, M * 64, d, qbar.device)
+    if out is None:
+        cap = capacity if capacity is not None else psa_route_capacity(B, H, M, causal)
+        out = (torch.empty(B * H * M + 1, dtype=torch.int32, device=qbar.device),
+               torch.empty(max(cap, 1), dtype=torch.int32, device=qbar.device),
+               torch.empty(1, dtype=torch.int32, device=qbar.device))
+    row_ptr, col_idx, nnz = out
+    _check("psa_route_thresh", lib().psa_route_thresh(
+        _ptr(qbar), _ptr(kbar), B, H, M, d, float(alpha), int(causal), int(keep_first), _ptr(row_ptr),
+        _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(ws), ws.numel(), _stream(stream)))
+    return row_ptr, col_idx, nnz
+
+
+def psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_size: int = 64,
+             ws=None, out=None, lse=None, want_lse: bool = False, stream=None):
+    """Returns out (bf16 [B,H,N,d]) and, if requested, lse (float32 [B,H,N])."""
+    B, H, N, d = _shape(q)
+    if ws is None:
+        ws = workspace(B, H, N, d, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    _check("psa_attn", lib().psa_attn(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+        B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return (out, lse) if lse is not None else out
+
+
+def psa_dense(q, k, v, causal: bool = False, ws=None, out=None, lse=None, want_lse: bool = False,
+              stream=None):
+    """Dense softmax attention through the same tensor-core kernel."""
+    B, H, N, d = _shape(q)
+    if ws is None:
+        ws = workspace(B, H, N, d, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    _check("psa_dense", lib().psa_dense(
+        _ptr(q), _ptr(k), _ptr(v), B, H, N, d, int(causal), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return (out, lse) if lse is not None else out
+
+
+def psa_read_status(ws, stream=None) -> int:
+    """Synchronise the stream and return the device status word of ``ws``."""
+    st = ctypes.c_int(-1)
+    _check("psa_read_status", lib().psa_read_status(_ptr(ws), ctypes.byref(st), _stream(stream)))
+    return int(st.value)
+
+
+def psa_forward(q, k, v, mode: str = "topk", density: float = 0.15, alpha: float = 0.5,
+                causal: bool = False, keep_first: bool = False, ws=None, stream=None):
+    """The whole path in one call (pool -> route -> attention), as the usage
+    line of the PISA summary calls it: f(q, k, v, density=0.15, block_size=64).
+    Returns (out, (row_ptr, col_idx, nnz))."""
+    B, H, N, d = _shape(q)
+    if ws is None:
+        ws = workspace(B, H, N, d, q.device)
+    qbar, kbar, vsum = psa_pool(q, k, v, stream=stream)
+    if mode == "topk":
+        csr = psa_route_topk(qbar, kbar, density, causal, stream=stream)
+    elif mode == "thresh":
+        csr = psa_route_thresh(qbar, kbar, alpha, causal, keep_first, ws=ws, stream=stream)
+    else:
+        raise ValueError("mode must be 'topk' or 'thresh'")
+    out = psa_attn(q, k, v, kbar, vsum, csr[0], csr[1], causal, ws=ws, stream=stream)
+    return out, csr

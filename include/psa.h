@@ -1,0 +1,187 @@
+/*
+ * psa.h -- C ABI of the B200 (sm_100a) block-sparse prefill attention library
+ * (PISA-style block routing with a 0th-order term for unselected blocks).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are row-major, contiguous.  Q, K, V and the output are
+ *    [B, H, N, d] bf16, passed as raw 16-bit patterns (psa_bf16_t).
+ *    Pooled statistics are [B, H, M, d] float32 with M = N / 64.
+ *    Block I of a head is tokens [64 I, 64 I + 64).
+ *  - Every pointer argument is a DEVICE pointer owned by the caller, except
+ *    where a comment says "host".  The library never allocates device memory
+ *    and never frees what it is given.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream) and returns a status code.
+ *  - Arguments are validated on the host before any launch: a bad argument
+ *    returns an error code and launches nothing.  Conditions that only the
+ *    device can see (a malformed block list, a bounded wait that ran out) are
+ *    recorded in the status word inside the caller's workspace; read it with
+ *    psa_read_status().
+ *  - Supported: block_size == 64, d in {64, 128}, N a positive multiple of
+ *    64, M = N / 64 <= 16384, B * H * N * d < 2^31.
+ *
+ * Rows of a block list ("CSR") are ordered (b, h, I) row-major: row
+ * r = (b * H + h) * M + I.  row_ptr has B*H*M + 1 int32 entries, col_idx
+ * holds the listed key blocks J of each row in ascending order.
+ *
+ * Citations name the web page and the section that defines the operation.
+ */
+#ifndef PSA_H
+#define PSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PSA_API __attribute__((visibility("default")))
+#else
+#define PSA_API
+#endif
+
+typedef uint16_t psa_bf16_t; /* raw bfloat16 bits */
+
+enum psa_status {
+    PSA_OK = 0,
+    PSA_ERR_ARG = 1,          /* null pointer, non-positive size, bad flag      */
+    PSA_ERR_SHAPE = 2,        /* N not a multiple of block_size, sizes too big */
+    PSA_ERR_UNSUPPORTED = 3,  /* block_size != 64, d not in {64, 128}, M > 16384 */
+    PSA_ERR_CAPACITY = 4,     /* workspace or col_idx capacity too small       */
+    PSA_ERR_CUDA = 5,         /* a CUDA runtime / driver call failed           */
+    PSA_ERR_TIMEOUT = 6,      /* device: a bounded wait ran out (kernel quit)   */
+    PSA_ERR_CSR = 7,          /* device: a listed block is out of range or repeated */
+    PSA_ERR_DEVICE = 8        /* no sm_100 device current                      */
+};
+
+/* Text for a status code (static storage, never NULL). */
+PSA_API const char* psa_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+PSA_API int psa_version(void);
+
+/*
+ * Bytes of device workspace that psa_route_thresh, psa_attn and psa_dense
+ * need for a problem of this shape (one workspace serves all three).  The
+ * workspace must be 256-byte aligned and is owned by the caller; calls that
+ * share one workspace must be ordered on one stream.  Returns 0 for invalid
+ * sizes.
+ */
+PSA_API size_t psa_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Worst-case number of listed blocks over all rows (the col_idx capacity
+ * that can never overflow): B*H*M*M, or B*H*M*(M+1)/2 when causal.
+ */
+PSA_API size_t psa_route_capacity(int B, int H, int M, int causal);
+
+/*
+ * a1. Pooling [PISA summary, "How are candidate blocks narrowed": a
+ * representative query and key per block and the sum of the values;
+ * FlashPrefill summary, 2.a "Block approximation": average-pooled keys].
+ *   qbar[b,h,I,:] = mean of q over block I     (float32, [B,H,M,d])
+ *   kbar[b,h,J,:] = mean of k over block J     (float32, [B,H,M,d])
+ *   vsum[b,h,J,:] = sum  of v over block J     (float32, [B,H,M,d])
+ * Accumulates in float32.  Errors: PSA_ERR_ARG, PSA_ERR_SHAPE,
+ * PSA_ERR_UNSUPPORTED, PSA_ERR_CUDA.
+ */
+PSA_API int psa_pool(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v,
+             int B, int H, int N, int d, int block_size,
+             float* qbar, float* kbar, float* vsum, void* stream);
+
+/*
+ * a2 + a3. Block scores and top-k routing [PISA summary, "How are candidate
+ * blocks narrowed" and usage line `density=0.15`].
+ *   s_IJ = qbar_I . kbar_J / sqrt(d) (float32), candidates J < M, or J <= I
+ *   when causal.  Row I keeps k = clamp(ceil(fl32(density * M)), 1, #cand)
+ *   blocks: the k highest scores, ties to the smaller J; when causal the
+ *   diagonal block takes one of the k slots and the other k-1 are the best
+ *   J < I.  Lists ascending.
+ * Outputs: row_ptr [B*H*M + 1], col_idx [capacity] (device int32) and
+ * *nnz_out (device int32) = total listed.  Errors: PSA_ERR_ARG,
+ * PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY (capacity below the exact total,
+ * which the host knows for top-k), PSA_ERR_CUDA.
+ */
+PSA_API int psa_route_topk(const float* qbar, const float* kbar,
+                   int B, int H, int M, int d, float density, int causal,
+                   int* row_ptr, int* col_idx, size_t capacity, int* nnz_out,
+                   void* stream);
+
+/*
+ * a2 + a4. Block scores and sorting-free threshold routing [FlashPrefill
+ * summary, 2.b "Max-based dynamic thresholding": thresh_I = alpha *
+ * max_J Score_IJ].  Keeps J iff s_IJ >= alpha * max over candidates
+ * (float32), plus the diagonal block I, plus block 0 when keep_first.
+ * Lists ascending.  The total is data dependent: *nnz_out (device) receives
+ * the exact total; if it exceeds `capacity`, rows past the capacity are cut
+ * (row_ptr stays a valid, truncated CSR) and the caller must retry with a
+ * larger col_idx.  psa_route_capacity() never overflows.
+ * `workspace` (device, psa_workspace_size(B,H,64*M,d) bytes) holds the row
+ * counts and bit masks between the three launches.  Errors: PSA_ERR_ARG,
+ * PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY (workspace too small), PSA_ERR_CUDA.
+ */
+PSA_API int psa_route_thresh(const float* qbar, const float* kbar,
+                     int B, int H, int M, int d, float alpha, int causal,
+                     int keep_first, int* row_ptr, int* col_idx, size_t capacity,
+                     int* nnz_out, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/*
+ * a5 - a7. Exact attention on the listed blocks plus the 0th-order term of
+ * every other candidate, in one softmax [PISA summary, routing table and
+ * "Why approximating unselected blocks keeps softmax intact"; FlashPrefill
+ * summary, 2.c "Index-driven physical jumping" for the addressing].
+ *   For query i of block I: z_ij = q_i.k_j / sqrt(d) over the tokens of the
+ *   listed blocks (causal: j <= i inside the diagonal block), and
+ *   a_iJ = q_i.kbar_J / sqrt(d) for each unlisted candidate J (causal:
+ *   J < I).  out_i = (sum e^z v_j + sum e^a vsum_J) /
+ *                    (sum e^z + 64 sum e^a),  lse_i = ln of that denominator
+ *   (natural log, including the common stabiliser).
+ * Inputs: q, k, v bf16 [B,H,N,d]; kbar, vsum float32 [B,H,M,d] from
+ * psa_pool; row_ptr / col_idx from a router or from the caller, where
+ * col_capacity is the number of int32 entries col_idx points to (a row whose
+ * row_ptr range leaves [0, col_capacity] is treated as empty and recorded as
+ * PSA_ERR_CSR, so the kernel never reads past the caller's buffer).
+ * Outputs: out bf16 [B,H,N,d]; lse float32 [B,H,N] (may be NULL).
+ * A malformed list entry is recorded as PSA_ERR_CSR in the workspace
+ * status: an entry out of range (J >= M, or J > I when causal) is skipped,
+ * a repeated entry is counted each time it appears.
+ * Errors: PSA_ERR_ARG, PSA_ERR_SHAPE, PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY
+ * (workspace too small), PSA_ERR_DEVICE, PSA_ERR_CUDA.
+ */
+PSA_API int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v,
+             const float* kbar, const float* vsum,
+             const int* row_ptr, const int* col_idx, size_t col_capacity,
+             int B, int H, int N, int d, int block_size, int causal,
+             psa_bf16_t* out, float* lse,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Dense attention (density = 1: every candidate block exact) through the
+ * same tensor-core kernel: the comparison baseline [PISA summary, "first
+ * check: compare dense and PISA outputs on the same seed and input";
+ * FlashAttention blog, section 1].  out = softmax(q k^T / sqrt(d)) v with
+ * the causal mask when `causal`.  Needs a workspace (it pools the keys to
+ * pick its softmax stabiliser).  Errors as psa_attn.
+ */
+PSA_API int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v,
+              int B, int H, int N, int d, int causal,
+              psa_bf16_t* out, float* lse,
+              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then copies the device status word of `workspace`
+ * into *status (host pointer): PSA_OK, or the first device-side error
+ * recorded since the last call that reset it (psa_route_thresh, psa_attn
+ * and psa_dense reset it at their start).  Returns PSA_OK or PSA_ERR_CUDA.
+ */
+PSA_API int psa_read_status(const void* workspace, int* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PSA_H */

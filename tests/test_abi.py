@@ -1,0 +1,105 @@
+"""CPU checks of the C-ABI library: it loads, exports every entry point that
+include/psa.h declares, and rejects bad arguments on the host (these calls
+return before any CUDA call, so they need no GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_psa_b200 import psa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = ctypes.c_void_p(1 << 20)   # a 16-byte-aligned address that is never dereferenced
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "psa.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"PSA_API\s+[\w\s\*]*?\b(psa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = declared_symbols()
+    for want in ("psa_pool", "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = psa.lib()
+    names = declared_symbols()
+    assert names
+    for name in names:
+        assert hasattr(L, name), name
+    assert set(psa.EXPORTS) == set(names)
+
+
+def test_status_strings():
+    for code in range(0, 9):
+        assert psa.status_text(code)
+    assert psa.status_text(PSA_UNKNOWN := 1234) == "unknown status"
+
+
+def test_workspace_and_capacity_sizes():
+    assert psa.psa_workspace_size(1, 12, 32768, 128) > 0
+    assert psa.psa_workspace_size(1, 12, 32768 + 1, 128) == 0      # ragged N
+    assert psa.psa_workspace_size(1, 12, 32768, 96) == 0            # unsupported d
+    assert psa.psa_route_capacity(1, 12, 512, False) == 12 * 512 * 512
+    assert psa.psa_route_capacity(1, 8, 2048, True) == 8 * 2048 * 2049 // 2
+    assert psa.psa_route_capacity(0, 8, 2048, True) == 0
+
+
+def test_host_validation_rejects_bad_arguments():
+    L = psa.lib()
+    S = ctypes.c_void_p(0)
+    # null pointers
+    assert L.psa_pool(None, FAKE, FAKE, 1, 1, 64, 64, 64, FAKE, FAKE, FAKE, S) == psa.PSA_ERR_ARG
+    # block size, head dim, ragged N
+    assert L.psa_pool(FAKE, FAKE, FAKE, 1, 1, 64, 64, 32, FAKE, FAKE, FAKE, S) == psa.PSA_ERR_UNSUPPORTED
+    assert L.psa_pool(FAKE, FAKE, FAKE, 1, 1, 64, 80, 64, FAKE, FAKE, FAKE, S) == psa.PSA_ERR_UNSUPPORTED
+    assert L.psa_pool(FAKE, FAKE, FAKE, 1, 1, 100, 64, 64, FAKE, FAKE, FAKE, S) == psa.PSA_ERR_SHAPE
+    assert L.psa_pool(FAKE, FAKE, FAKE, 0, 1, 64, 64, 64, FAKE, FAKE, FAKE, S) == psa.PSA_ERR_ARG
+    # misaligned tensor
+    assert L.psa_pool(ctypes.c_void_p((1 << 20) + 2), FAKE, FAKE, 1, 1, 64, 64, 64, FAKE, FAKE, FAKE, S) \
+        == psa.PSA_ERR_ARG
+    # top-k: capacity below the exact total, bad density
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 2 * 16 * 4 - 1, FAKE, S) \
+        == psa.PSA_ERR_CAPACITY
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, float("nan"), 0, FAKE, FAKE, 1 << 20, FAKE, S) \
+        == psa.PSA_ERR_ARG
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 2, FAKE, FAKE, 1 << 20, FAKE, S) == psa.PSA_ERR_ARG
+    # threshold: workspace too small, bad alpha
+    assert L.psa_route_thresh(FAKE, FAKE, 1, 2, 16, 64, 0.5, 0, 0, FAKE, FAKE, 1 << 20, FAKE, FAKE, 16, S) \
+        == psa.PSA_ERR_CAPACITY
+    assert L.psa_route_thresh(FAKE, FAKE, 1, 2, 16, 64, float("inf"), 0, 0, FAKE, FAKE, 1 << 20, FAKE, FAKE,
+                              1 << 30, S) == psa.PSA_ERR_ARG
+    # attention: workspace too small, misaligned workspace, M too large
+    ws = psa.psa_workspace_size(1, 2, 1024, 64)
+    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 1, 2, 1024, 64, 64, 0, FAKE, None, FAKE,
+                      ws - 1, S) == psa.PSA_ERR_CAPACITY
+    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 1, 2, 1024, 64, 64, 0, FAKE, None,
+                      ctypes.c_void_p((1 << 20) + 16), ws, S) == psa.PSA_ERR_ARG
+    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 1, 1, 64 * 16385, 64, 64, 0, FAKE, None,
+                      FAKE, 1 << 40, S) == psa.PSA_ERR_UNSUPPORTED
+    assert L.psa_dense(FAKE, FAKE, FAKE, 1, 2, 1024, 64, 3, FAKE, None, FAKE, ws, S) == psa.PSA_ERR_ARG
+    assert L.psa_read_status(None, None, S) == psa.PSA_ERR_ARG
+
+
+def test_binding_names_match_c_entry_points():
+    for name in ("psa_pool", "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense",
+                 "psa_workspace_size", "psa_route_capacity", "psa_read_status"):
+        assert callable(getattr(psa, name))
+
+
+def test_no_cpu_fallback_in_product_package():
+    """The product package never imports the oracle."""
+    pkg = os.path.join(ROOT, "block_sparse_attention_psa_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(dirpath, fn)) as f:
+                    src = f.read()
+                assert "oracle" not in re.sub(r"#.*|//.*", "", src).replace("oracle.", "ORACLE") or \
+                    "import oracle" not in src, fn
+                assert "import oracle" not in src and "from oracle" not in src, fn

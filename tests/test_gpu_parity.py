@@ -1,0 +1,199 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small cases run the oracle on every unit; the full-size workloads run the
+GPU exactly as ``bench.py`` launches it and compare every block list plus a
+seeded sample of query blocks."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.psa_oracle as O
+from block_sparse_attention_psa_b200 import psa
+from block_sparse_attention_psa_b200.inputs import WORKLOADS, make_qkv, workload_inputs
+from tests.parity import (check_output, check_pool, check_routing, f64, run_gpu, sample_units)
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(q, k, v, mode, param, causal=False, keep_first=False, units=None):
+    g = run_gpu(q, k, v, mode, param, causal, keep_first)
+    assert g["status"] == psa.PSA_OK, psa.status_text(g["status"])
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    s = O.block_scores(qbar, kbar)
+    check_routing(g, s, mode, param, causal, keep_first)
+    return check_output(g, q, k, v, kbar, vsum, causal, units)
+
+
+# ------------------------------------------------------------------ small, every unit
+def test_tiny_iid_topk_quarter():
+    q, k, v = workload_inputs("tiny_iid_n1k")
+    _full_check(q, k, v, "topk", 0.25)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_clustered_topk_ragged(d, causal):
+    # M = 37: an odd block count (half-empty exact tile, partial pooled tile)
+    q, k, v = make_qkv(2, 2, 37 * 64, d, "clustered", seed=3)
+    _full_check(q, k, v, "topk", 0.15, causal)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal,keep_first", [(False, False), (True, True), (True, False)])
+def test_clustered_threshold(d, causal, keep_first):
+    q, k, v = make_qkv(1, 3, 45 * 64, d, "clustered_slash", seed=4)
+    _full_check(q, k, v, "thresh", 0.5, causal, keep_first)
+
+
+def test_many_pooled_tiles():
+    # M = 300 > 2 * 128: several pooled-key tiles per unit, ragged last tile
+    q, k, v = make_qkv(1, 1, 300 * 64, 64, "clustered", seed=5)
+    B, H, N, d = q.shape
+    g = run_gpu(q, k, v, "topk", 0.05)
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    check_routing(g, O.block_scores(qbar, kbar), "topk", 0.05, False)
+    check_output(g, q, k, v, kbar, vsum, False, sample_units(B, H, N // 64, 40, seed=1, g=g))
+
+
+def test_single_block():
+    q, k, v = make_qkv(1, 2, 64, 128, "iid", seed=6)
+    for causal in (False, True):
+        _full_check(q, k, v, "topk", 0.5, causal)
+
+
+@pytest.mark.parametrize("density", [0.0, 1.0])
+def test_topk_extremes(density):
+    q, k, v = make_qkv(1, 2, 20 * 64, 64, "iid", seed=7)
+    _full_check(q, k, v, "topk", density, False)
+
+
+# ------------------------------------------------------------------ dense path
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_dense_equals_softmax_attention(d, causal):
+    q, k, v = make_qkv(1, 2, 9 * 64, d, "iid", seed=8)
+    dq, dk, dv = (x.cuda() for x in (q, k, v))
+    out, lse = psa.psa_dense(dq, dk, dv, causal, want_lse=True)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(f64(q)), torch.from_numpy(f64(k)), torch.from_numpy(f64(v)), is_causal=causal)
+    err = np.abs(f64(out) - ref.numpy())
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
+    logits = torch.from_numpy(f64(q)) @ torch.from_numpy(f64(k)).transpose(-1, -2) / np.sqrt(d)
+    if causal:
+        n = q.shape[2]
+        logits = logits.masked_fill(torch.ones(n, n).triu(1).bool(), float("-inf"))
+    ref_lse = torch.logsumexp(logits, -1).numpy()
+    assert np.abs(f64(lse) - ref_lse).max() <= 1e-3 * max(1.0, np.abs(ref_lse).max())
+
+
+def test_tiny_density_one_equals_dense():
+    q, k, v = workload_inputs("tiny_iid_n1k")
+    g = run_gpu(q, k, v, "topk", 1.0)
+    dq, dk, dv = (x.cuda() for x in (q, k, v))
+    dense = psa.psa_dense(dq, dk, dv, False)
+    err = np.abs(f64(g["out"]) - f64(dense))
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3
+
+
+# ------------------------------------------------------------------ hand-built block lists
+def _attn_with_lists(q, k, v, lists, causal):
+    dq, dk, dv = (x.cuda() for x in (q, k, v))
+    B, H, N, d = q.shape
+    qbar, kbar, vsum = psa.psa_pool(dq, dk, dv)
+    rp, ci = O._to_csr(lists)
+    rp_t = torch.tensor(rp, dtype=torch.int32, device="cuda")
+    ci_t = torch.tensor(ci if ci.size else [0], dtype=torch.int32, device="cuda")
+    ws = psa.workspace(B, H, N, d)
+    out, lse = psa.psa_attn(dq, dk, dv, kbar, vsum, rp_t, ci_t, causal, ws=ws, want_lse=True)
+    status = psa.psa_read_status(ws)
+    return dict(out=out.cpu(), lse=lse.cpu(), row_ptr=rp, col_idx=ci, status=status,
+                kbar=kbar.cpu(), vsum=vsum.cpu())
+
+
+def test_empty_lists_are_pure_zeroth_order():
+    q, k, v = make_qkv(1, 2, 12 * 64, 128, "clustered", seed=9)
+    lists = [np.zeros(0, dtype=np.int64) for _ in range(2 * 12)]
+    g = _attn_with_lists(q, k, v, lists, False)
+    assert g["status"] == psa.PSA_OK
+    _, kbar, vsum = O.pool(f64(q), f64(k), f64(v))
+    check_output(g, q, k, v, kbar, vsum, False)
+
+
+def test_random_lists_every_size():
+    rng = np.random.default_rng(10)
+    q, k, v = make_qkv(1, 2, 23 * 64, 64, "clustered", seed=11)
+    for causal in (False, True):
+        lists = []
+        for _ in range(2):
+            for I in range(23):
+                n = I + 1 if causal else 23
+                keep = rng.random(n) < rng.random()
+                if causal:
+                    keep[I] = True
+                lists.append(np.nonzero(keep)[0])
+        g = _attn_with_lists(q, k, v, lists, causal)
+        assert g["status"] == psa.PSA_OK
+        _, kbar, vsum = O.pool(f64(q), f64(k), f64(v))
+        check_output(g, q, k, v, kbar, vsum, causal)
+
+
+def test_malformed_list_is_reported_not_fatal():
+    q, k, v = make_qkv(1, 1, 8 * 64, 64, "iid", seed=12)
+    lists = [np.array([0, 1])] * 7 + [np.array([3, 99])]   # J = 99 is out of range
+    g = _attn_with_lists(q, k, v, lists, False)
+    assert g["status"] == psa.PSA_ERR_CSR
+    # the device is still healthy afterwards
+    g2 = _attn_with_lists(q, k, v, [np.array([0, 1])] * 8, False)
+    assert g2["status"] == psa.PSA_OK
+
+
+def test_huge_logit_goes_through_exact_fixup():
+    # one key whose logit exceeds its block mean by ~95: the fixed stabiliser
+    # overflows there, and the exact fixup path must take over for that row
+    B, H, N, d = 1, 1, 4 * 64, 64
+    q = torch.zeros(B, H, N, d)
+    k = torch.zeros(B, H, N, d)
+    v = torch.randn(B, H, N, d, generator=torch.Generator().manual_seed(13))
+    q[..., 0] = 8.0
+    k[0, 0, 70, 0] = 100.0
+    q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+    lists = [np.array([0, 1, 2, 3])] * 4
+    g = _attn_with_lists(q, k, v, lists, False)
+    assert g["status"] == psa.PSA_OK
+    _, kbar, vsum = O.pool(f64(q), f64(k), f64(v))
+    check_output(g, q, k, v, kbar, vsum, False)
+
+
+# ------------------------------------------------------------------ full-size workloads
+def _full_size(name, density=None, n_units=48):
+    w = WORKLOADS[name]
+    q, k, v = workload_inputs(name)
+    mode, param = w["routing"]
+    if density is not None:
+        param = density
+    g = run_gpu(q, k, v, mode, param, w["causal"], w["keep_first"])
+    assert g["status"] == psa.PSA_OK
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    s = O.block_scores(qbar, kbar)
+    check_routing(g, s, mode, param, w["causal"], w["keep_first"])
+    M = w["N"] // 64
+    units = sample_units(w["B"], w["H"], M, n_units, seed=2, g=g)
+    return check_output(g, q, k, v, kbar, vsum, w["causal"], units)
+
+
+def test_full_dit_video_topk():
+    _full_size("dit_video_n32k")
+
+
+def test_full_dit_video_threshold():
+    _full_size("dit_video_n32k_thresh")
+
+
+def test_full_long_causal_threshold():
+    _full_size("long_causal_n128k", n_units=40)
+
+
+@pytest.mark.parametrize("density", [0.05, 1.0])
+def test_full_sweep(density):
+    _full_size("sweep_n64k", density=density, n_units=40)
