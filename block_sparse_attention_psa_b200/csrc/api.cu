@@ -20,7 +20,7 @@ WorkspaceLayout workspace_layout(long long BH, long long M, long long d) {
   o += align256(static_cast<size_t>(BH * M) * 4);
   L.kbar_bf16 = o;
   o += align256(static_cast<size_t>(BH * M * d) * 2);
-  L.vbar_bf16 = o;
+  L.vsum_bf16 = o;
   o += align256(static_cast<size_t>(BH * M * d) * 2);
   L.row_count = o;
   o += align256(static_cast<size_t>(BH * M) * 4);
@@ -215,7 +215,7 @@ int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, cons
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
   if (e != cudaSuccess) return PSA_ERR_CUDA;
   uint16_t* kb16 = reinterpret_cast<uint16_t*>(ws + L.kbar_bf16);
-  uint16_t* vb16 = reinterpret_cast<uint16_t*>(ws + L.vbar_bf16);
+  uint16_t* vb16 = reinterpret_cast<uint16_t*>(ws + L.vsum_bf16);
   e = psa::launch_stats_to_bf16(kbar, vsum, bh * M * d, kb16, vb16, st);
   if (e != cudaSuccess) return PSA_ERR_CUDA;
   psa::AttnLaunch a;
@@ -223,7 +223,7 @@ int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, cons
   a.k = k;
   a.v = v;
   a.kbar_bf16 = kb16;
-  a.vbar_bf16 = vb16;
+  a.vsum_bf16 = vb16;
   a.kbar32 = kbar;
   a.vsum32 = vsum;
   a.row_ptr = row_ptr;
@@ -270,7 +270,7 @@ int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int
   a.k = k;
   a.v = v;
   a.kbar_bf16 = kb16;
-  a.vbar_bf16 = kb16;
+  a.vsum_bf16 = kb16;
   a.out = out;
   a.lse = lse;
   a.BH = static_cast<int>(bh);

@@ -41,7 +41,11 @@
 namespace psa {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;     // WG0: TMA producers (warps 0, 2), MMA issuers (warps 1, 3); WG1, WG2: softmax
+constexpr int kRegsProducer = 56;  // setmaxnreg split: 128 x 56 + 256 x 224 = 384 x 168
+constexpr int kRegsSoftmax = 224;
+constexpr int kRegsLaunch = 168;
+constexpr int kColCache = 1024;   // listed blocks of a unit kept in shared memory
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D>
@@ -51,16 +55,16 @@ struct Cfg {
   static constexpr int kKVBytes = 128 * D * 2;   // two key blocks
   static constexpr int kPBytes = 128 * 64 * 2;   // P^T tile
   static constexpr int kOutBytes = 64 * D * 2;   // output staging
-  static constexpr int kNQ = 2, kNK = 2, kNV = 2, kNP = 2;
+  static constexpr int kNQ = 2, kNK = 2, kNV = 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kNQ * kQBytes;
   static constexpr int kOffV = kOffK + kNK * kKVBytes;
-  static constexpr int kOffP = kOffV + kNV * kKVBytes;
-  static constexpr int kOffOut = kOffP + kNP * kPBytes;
+  static constexpr int kOffP = kOffV + kNV * kKVBytes;   // one P^T tile per softmax warpgroup
+  static constexpr int kOffOut = kOffP + 2 * kPBytes;
   static constexpr int kOffMisc = kOffOut + kOutBytes;
-  // misc: 32 barriers (256 B) + tmem slot / flags (256 B) + red[4][64] +
-  // c2[64] + invl[64] + l[64] + bitmap[kMaxBlocks / 32]
-  static constexpr int kMiscBytes = 256 + 256 + 4 * 64 * 4 + 3 * 64 * 4 + kMaxBlocks / 8;
+  // misc: 32 barriers (256 B) + tmem slot / flags (256 B) + red[8][64] f32 +
+  // c2[64] + invl[64] + l[64] + bitmap[kMaxBlocks / 32] + cols[kColCache]
+  static constexpr int kMiscBytes = 256 + 256 + 8 * 64 * 4 + 3 * 64 * 4 + kMaxBlocks / 8 + kColCache * 4;
   static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
   // kind::f16, bf16 x bf16 -> f32.  GEMM1: M=128 keys, N=64 queries, both
   // K-major.  GEMM2: M=128 (feature rows), N=64 queries, both MN-major.
@@ -89,8 +93,10 @@ struct Unit {
 
 __device__ __forceinline__ Unit make_unit(int u, const Params& p) {
   Unit x;
-  x.I = p.M - 1 - u / p.BH;  // largest I first (causal rows are the longest)
-  x.bh = u % p.BH;
+  // head-major, largest I first inside a head: concurrent CTAs share one
+  // head's K/V in L2, and long causal rows are scheduled first
+  x.bh = u / p.M;
+  x.I = p.M - 1 - (u - x.bh * p.M);
   x.row = x.bh * p.M + x.I;
   x.cand = p.causal ? x.I + 1 : p.M;   // exact candidates J < cand
   x.pcand = p.causal ? x.I : p.M;      // 0th-order candidates J < pcand
@@ -141,13 +147,13 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Column reduction over the 128 softmax threads: v[64] per thread,
+// Column reduction over the 256 softmax threads (8 warps): v[64] per thread,
 // out[q] = sum (or max) over threads of v[q].  Butterfly transpose-reduce
 // inside each warp (after it, lane L holds columns 2*rev5(L) and +1), then
-// the four warps combine through shared memory.
+// the eight warps combine through shared memory.
 template <bool kMax>
-__device__ __forceinline__ void group_reduce64(float (&v)[64], float* red, float* out, int lane, int wq,
-                                               int tid) {
+__device__ __forceinline__ void group_reduce64(float (&v)[64], float* red, float* out, int lane, int gwarp,
+                                               int gtid) {
 #pragma unroll
   for (int step = 0; step < 5; ++step) {
     const int o = 16 >> step;
@@ -163,14 +169,25 @@ __device__ __forceinline__ void group_reduce64(float (&v)[64], float* red, float
   }
   const int col = ((lane & 16) ? 32 : 0) + ((lane & 8) ? 16 : 0) + ((lane & 4) ? 8 : 0) +
                   ((lane & 2) ? 4 : 0) + ((lane & 1) ? 2 : 0);
-  red[wq * 64 + col] = v[0];
-  red[wq * 64 + col + 1] = v[1];
-  named_barrier_sync(1, 128);
-  if (tid < 64) {
-    const float a = red[tid], b = red[64 + tid], c = red[128 + tid], d = red[192 + tid];
-    out[tid] = kMax ? fmaxf(fmaxf(a, b), fmaxf(c, d)) : (a + b) + (c + d);
+  red[gwarp * 64 + col] = v[0];
+  red[gwarp * 64 + col + 1] = v[1];
+  named_barrier_sync(1, 256);
+  if (gtid < 64) {
+    float r = red[gtid];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) r = kMax ? fmaxf(r, red[w * 64 + gtid]) : r + red[w * 64 + gtid];
+    out[gtid] = r;
   }
-  named_barrier_sync(1, 128);
+  named_barrier_sync(1, 256);
+}
+
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
 }
 
 template <int D>
@@ -187,28 +204,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sP = smem + C::kOffP;
   uint8_t* sOut = smem + C::kOffOut;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffMisc);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 2;
-  uint64_t* k_full = bars + 4;
-  uint64_t* k_empty = bars + 6;
-  uint64_t* v_full = bars + 8;
-  uint64_t* v_empty = bars + 10;
-  uint64_t* s_full = bars + 12;
-  uint64_t* s_empty = bars + 14;
-  uint64_t* p_full = bars + 16;
-  uint64_t* p_empty = bars + 18;
-  uint64_t* o_full = bars + 20;
-  uint64_t* o_empty = bars + 22;
-  uint64_t* drain = bars + 24;
+  // Rings are indexed by the parity of the running tile index: K stage,
+  // S^T buffer, V stage and P^T buffer b all serve the tiles of parity b.
+  uint64_t* q_full = bars + 0;    // Q landed                      (TMA)
+  uint64_t* q_empty = bars + 2;   // last GEMM1 of the unit done   (commit)
+  uint64_t* k_full = bars + 4;    // K tile landed                 (TMA)
+  uint64_t* s_full = bars + 6;    // GEMM1 done: S^T ready, K stage free (commit)
+  uint64_t* s_empty = bars + 8;   // S^T read by the softmax       (4 warps)
+  uint64_t* v_full = bars + 10;   // V tile landed                 (TMA)
+  uint64_t* p_full = bars + 12;   // P^T written                   (4 warps)
+  uint64_t* g2_done = bars + 14;  // GEMM2 done: V stage and P^T buffer free (commit)
+  uint64_t* o_full = bars + 16;   // last GEMM2 of the unit done   (commit)
+  uint64_t* o_empty = bars + 18;  // O^T read by the epilogue      (8 warps)
+  uint64_t* drain = bars + 20;    // [2] teardown of the two issuers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* unit_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   volatile int* stop_s = reinterpret_cast<volatile int*>(tmem_slot + 3);
   float* red = reinterpret_cast<float*>(smem + C::kOffMisc + 512);
-  float* c2s = red + 256;
+  float* c2s = red + 8 * 64;
   float* invl = c2s + 64;
   float* lsh = invl + 64;
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(lsh + 64);
+  int* cols = reinterpret_cast<int*>(bitmap + kMaxBlocks / 32);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -217,17 +235,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
-      mbar_init(&p_full[i], 128);
-      mbar_init(&p_empty[i], 1);
+      mbar_init(&s_empty[i], 4);   // one arrival per softmax warp
+      mbar_init(&v_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&g2_done[i], 1);
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], 128);
+      mbar_init(&o_empty[i], 8);
+      mbar_init(&drain[i], 1);
     }
-    mbar_init(drain, 1);
     *abort_flag = 0;
     *unit_flag = 0;
     fence_barrier_init();
@@ -248,15 +264,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    int kc = 0, vc = 0, qc = 0;  // loads issued (lane 0's counts)
+  if (warp < 4) {
+  reg_dealloc<kRegsProducer>();
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers
+    // warp 0: Q and the key tiles (GEMM1 operand A); warp 2: the value tiles
+    // (GEMM2 operand A).  Separate warps, so a value stage still held by a
+    // GEMM2 never delays the next key prefetch.
+    const bool keys = warp == 0;
+    int sc = 0;              // running tile index
+    int ld[2] = {0, 0};      // loads issued into each stage (lane 0)
+    int qc = 0;
     bool ok = true;
     int ul = 0;
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ul) {
       const Unit x = make_unit(u, p);
       const int qb = ul & 1;
-      if (lane == 0) {
+      if (keys && lane == 0) {
         ok = mbar_wait(&q_empty[qb], ((ul >> 1) & 1) ^ 1, abort_flag, p.status);
         if (ok) {
           mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
@@ -268,15 +292,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       int colv = 0;
-      for (int t = 0; t < x.ntiles && ok; ++t) {
+      for (int t = 0; t < x.ntiles && ok; ++t, ++sc) {
         int kind, ti;
         tile_kind(x, t, kind, ti);
+        if (!keys && kind == 0) continue;  // pooled-key max tiles have no value operand
         int y0, y1;
-        const CUtensorMap* mk;
-        const CUtensorMap* mv;
+        const CUtensorMap* m;
         if (kind == 2) {
-          mk = &tmK;
-          mv = &tmV;
+          m = keys ? &tmK : &tmV;
           const int e2 = 2 * ti;
           int j1, j2;
           if (p.dense) {
@@ -296,37 +319,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           y0 = 64 * j1;
           y1 = 64 * j2;
         } else {
-          mk = &tmKb;
-          mv = &tmVb;
+          m = keys ? &tmKb : &tmVb;
           y0 = 128 * ti;
           y1 = y0 + 64;
         }
         if (lane == 0) {
-          const int ks = kc % C::kNK;
-          ok = mbar_wait(&k_empty[ks], ((kc / C::kNK) & 1) ^ 1, abort_flag, p.status);
+          const int st = sc & 1;
+          // the stage is free once the GEMM that read its previous contents is done
+          ok = mbar_wait(keys ? &s_full[st] : &g2_done[st], (ld[st] & 1) ^ 1, abort_flag, p.status);
           if (ok) {
-            mbar_arrive_expect_tx(&k_full[ks], C::kKVBytes);
-            uint8_t* dst = sK + ks * C::kKVBytes;
+            uint64_t* full = keys ? &k_full[st] : &v_full[st];
+            mbar_arrive_expect_tx(full, C::kKVBytes);
+            uint8_t* dst = (keys ? sK : sV) + st * C::kKVBytes;
 #pragma unroll
             for (int c = 0; c < C::kChunks; ++c) {
-              tma_load_3d(mk, dst + c * 16384, &k_full[ks], 64 * c, y0, x.bh);
-              tma_load_3d(mk, dst + c * 16384 + 8192, &k_full[ks], 64 * c, y1, x.bh);
+              tma_load_3d(m, dst + c * 16384, full, 64 * c, y0, x.bh);
+              tma_load_3d(m, dst + c * 16384 + 8192, full, 64 * c, y1, x.bh);
             }
-            ++kc;
-          }
-          if (ok && kind != 0) {
-            const int vs = vc % C::kNV;
-            ok = mbar_wait(&v_empty[vs], ((vc / C::kNV) & 1) ^ 1, abort_flag, p.status);
-            if (ok) {
-              mbar_arrive_expect_tx(&v_full[vs], C::kKVBytes);
-              uint8_t* dst = sV + vs * C::kKVBytes;
-#pragma unroll
-              for (int c = 0; c < C::kChunks; ++c) {
-                tma_load_3d(mv, dst + c * 16384, &v_full[vs], 64 * c, y0, x.bh);
-                tma_load_3d(mv, dst + c * 16384 + 8192, &v_full[vs], 64 * c, y1, x.bh);
-              }
-              ++vc;
-            }
+            ++ld[st];
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -334,117 +344,126 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) {
       // make sure no bulk copy is still writing shared memory when we leave
-      for (int i = max(0, kc - C::kNK); i < kc; ++i) mbar_drain(&k_full[i % C::kNK], (i / C::kNK) & 1);
-      for (int i = max(0, vc - C::kNV); i < vc; ++i) mbar_drain(&v_full[i % C::kNV], (i / C::kNV) & 1);
+      for (int st = 0; st < 2; ++st)
+        if (ld[st] > 0) mbar_drain(keys ? &k_full[st] : &v_full[st], (ld[st] - 1) & 1);
       for (int i = max(0, qc - C::kNQ); i < qc; ++i) mbar_drain(&q_full[i % C::kNQ], (i / C::kNQ) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ GEMM1 issuer
+    // S^T[tile parity] = K_tile . Q^T for every tile, in order.
     if (lane == 0) {
-      int kc = 0, vc = 0, sc = 0, pc = 0;
+      static_assert(C::kNK == 2 && C::kNV == 2 && C::kNQ == 2, "rings alternate two stages");
+      const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      constexpr uint64_t kKVStep = C::kKVBytes >> 4, kQStep = C::kQBytes >> 4;  // 16-byte units
+      int sc = 0;
       bool ok = true;
-      bool pend = false, pend_first = false, pend_last = false;
-      int pend_ob = 0;
-      uint32_t pend_opar = 0;
-      auto issue_gemm2 = [&]() -> bool {
-        const int vs = vc % C::kNV, pb = pc & 1;
-        if (!mbar_wait(&v_full[vs], (vc / C::kNV) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(&p_full[pb], (pc >> 1) & 1, abort_flag, p.status)) return false;
-        if (pend_first && !mbar_wait(&o_empty[pend_ob], pend_opar, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint32_t va = smem_u32(sV + vs * C::kKVBytes);
-        const uint32_t pa = smem_u32(sP + pb * C::kPBytes);
-        const uint32_t dt = tbase + 128 + 64 * pend_ob;
-        // A = V tile viewed MN-major (feature atoms 16 KB apart; for d = 64
-        // the second atom repeats the first and its rows are never read)
-        const uint32_t lbo = D == 128 ? 16384 : 0;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc_mma_bf16(dt, sdesc_sw128(va + kk * 2048, lbo, 1024), sdesc_sw128(pa + kk * 2048, 16, 1024),
-                      C::kIdesc2, (pend_first && kk == 0) ? 0u : 1u);
-        tc_commit(&v_empty[vs]);
-        tc_commit(&p_empty[pb]);
-        if (pend_last) tc_commit(&o_full[pend_ob]);
-        ++vc;
-        ++pc;
-        return true;
-      };
       int ul = 0;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ul) {
         const Unit x = make_unit(u, p);
         const int qb = ul & 1;
         if (!(ok = mbar_wait(&q_full[qb], (ul >> 1) & 1, abort_flag, p.status))) break;
-        const uint32_t qa = smem_u32(sQ + qb * C::kQBytes);
-        const int g2_total = x.n_a2 + x.n_e;
-        int g2_seen = 0;
-        for (int t = 0; t < x.ntiles; ++t) {
-          int kind, ti;
-          tile_kind(x, t, kind, ti);
-          const int ks = kc % C::kNK, sb = sc & 1;
-          if (!(ok = mbar_wait(&k_full[ks], (kc / C::kNK) & 1, abort_flag, p.status))) break;
+        const uint64_t dq = dQ0 + qb * kQStep;
+        for (int t = 0; t < x.ntiles; ++t, ++sc) {
+          const int sb = sc & 1;
+          if (!(ok = mbar_wait(&k_full[sb], (sc >> 1) & 1, abort_flag, p.status))) break;
           if (!(ok = mbar_wait(&s_empty[sb], ((sc >> 1) & 1) ^ 1, abort_flag, p.status))) break;
           tc_fence_after();
-          const uint32_t ka = smem_u32(sK + ks * C::kKVBytes);
+          const uint64_t a = dK0 + sb * kKVStep;
           const uint32_t dt = tbase + 64 * sb;
+          tc_mma_bf16(dt, a, dq, C::kIdesc1, 0u);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            tc_mma_bf16(dt, sdesc_sw128(ka + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                        sdesc_sw128(qa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), C::kIdesc1,
-                        kk > 0 ? 1u : 0u);
-          tc_commit(&k_empty[ks]);
+          for (int kk = 1; kk < D / 16; ++kk)
+            tc_mma_bf16(dt, a + (kk >> 2) * 1024 + (kk & 3) * 2, dq + (kk >> 2) * 512 + (kk & 3) * 2,
+                        C::kIdesc1, 1u);
           tc_commit(&s_full[sb]);
           if (t == x.ntiles - 1) tc_commit(&q_empty[qb]);
-          ++kc;
-          ++sc;
-          if (pend) {
-            pend = false;
-            if (!(ok = issue_gemm2())) break;
-          }
-          if (kind != 0) {
-            pend = true;
-            pend_ob = ul & 1;
-            pend_opar = ((ul >> 1) & 1) ^ 1;
-            pend_first = g2_seen == 0;
-            pend_last = g2_seen == g2_total - 1;
-            ++g2_seen;
-          }
         }
       }
-      if (ok && pend) ok = issue_gemm2();
-      // every MMA issued so far must finish before TMEM is freed
-      tc_commit(drain);
-      mbar_drain(drain, 0);
+      // every MMA this thread issued must finish before TMEM is freed
+      tc_commit(&drain[0]);
+      mbar_drain(&drain[0], 0);
     }
     __syncwarp();
   } else {
+    // ------------------------------------------------------------ GEMM2 issuer
+    // O^T[unit parity] += V_tile^T . P^T for every A2 / E tile, in order.
+    if (lane == 0) {
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), D == 128 ? 16384 : 0, 1024);
+      // V viewed MN-major: feature atoms 16 KB apart (d = 64: the second
+      // atom repeats the first and its output rows are never read)
+      const uint64_t dP0 = sdesc_sw128(smem_u32(sP), 16, 1024);
+      constexpr uint64_t kKVStep = C::kKVBytes >> 4, kPStep = C::kPBytes >> 4;
+      int sc = 0;
+      int used[2] = {0, 0};  // GEMM2s issued on each buffer parity
+      bool ok = true;
+      int ul = 0;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ul) {
+        const Unit x = make_unit(u, p);
+        const int ob = ul & 1;
+        sc += x.n_a1;
+        const int g2_total = x.n_a2 + x.n_e;
+        for (int g = 0; g < g2_total; ++g, ++sc) {
+          const int pb = sc & 1;
+          const int n = pb ? used[1] : used[0];
+          if (!(ok = mbar_wait(&v_full[pb], n & 1, abort_flag, p.status))) break;
+          if (!(ok = mbar_wait(&p_full[pb], n & 1, abort_flag, p.status))) break;
+          if (g == 0 && !(ok = mbar_wait(&o_empty[ob], ((ul >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          const uint64_t a = dV0 + pb * kKVStep, b = dP0 + pb * kPStep;
+          const uint32_t dt = tbase + 128 + 64 * ob;
+          tc_mma_bf16(dt, a, b, C::kIdesc2, g == 0 ? 0u : 1u);
+#pragma unroll
+          for (int kk = 1; kk < 8; ++kk) tc_mma_bf16(dt, a + 128 * kk, b + 128 * kk, C::kIdesc2, 1u);
+          tc_commit(&g2_done[pb]);
+          if (g == g2_total - 1) tc_commit(&o_full[ob]);
+          if (pb) ++used[1]; else ++used[0];
+        }
+      }
+      tc_commit(&drain[1]);
+      mbar_drain(&drain[1], 0);
+    }
+    __syncwarp();
+  }
+  } else {
+    reg_alloc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax + epilogue
-    const int wq = warp & 3;             // TMEM lane quarter of this warp
-    const int trow = wq * 32 + lane;     // TMEM lane: key row of S^T, feature row of O^T
-    const int tid = threadIdx.x - 64;    // 0..127 inside the group
+    // Two warpgroups; warpgroup w handles the tiles whose running index has
+    // parity w (its own S^T TMEM buffer and P^T smem buffer).
+    const int w = (warp >> 2) - 1;
+    const int wq = warp & 3;              // TMEM lane quarter of this warp
+    const int trow = wq * 32 + lane;      // TMEM lane: key row of S^T, feature row of O^T
+    const int gtid = threadIdx.x - 128;   // 0..255 over both warpgroups
+    const int gwarp = gtid >> 5;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_addr = tbase + lane_addr + 64 * w;
+    uint8_t* prow = sP + w * C::kPBytes + trow * 128;
     float acc[64];   // running max in A1, then minus the stabiliser (log2 units)
-    float lsum[64];  // per-thread partial denominators
+    float lsum[64];  // this thread's share of the denominators
     // Waits in this group never leave the control flow: after a timeout
     // (abort raised) they return at once and the group runs on with garbage
-    // data until the next unit boundary, where all 128 threads take the same
+    // data until the next unit boundary, where all 256 threads take the same
     // stop decision.  This keeps every named barrier matched.
-    int sc = 0, pc = 0;
+    int sc = 0;   // running tile index (both warpgroups count every tile)
+    int my = 0;   // tiles of this warpgroup so far (S buffer phase)
+    int mp = 0;   // P^T tiles written by this warpgroup so far (P buffer phase)
     int ul = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++ul) {
-      named_barrier_sync(1, 128);
-      if (tid == 0) *stop_s = *abort_flag;
-      named_barrier_sync(1, 128);
+      named_barrier_sync(1, 256);
+      if (gtid == 0) *stop_s = *abort_flag;
+      named_barrier_sync(1, 256);
       if (*stop_s) break;
       const Unit x = make_unit(u, p);
       if (!p.dense) {
-        // mark the listed blocks (A2 skips them) and validate the list
+        // mark the listed blocks (A2 skips them), cache the list, validate it
         const int nw = (x.cand + 31) / 32;
-        for (int w = tid; w < nw; w += 128) bitmap[w] = 0u;
-        named_barrier_sync(1, 128);
+        for (int i = gtid; i < nw; i += 256) bitmap[i] = 0u;
+        named_barrier_sync(1, 256);
         bool bad = x.bad;
-        for (int i = tid; i < x.nsel; i += 128) {
+        for (int i = gtid; i < x.nsel; i += 256) {
           const int J = __ldg(p.col_idx + x.rp + i);
+          if (i < kColCache) cols[i] = J;
           if (J < 0 || J >= x.cand) {
             bad = true;
           } else {
@@ -453,129 +472,137 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (bad) record_status(p.status, kStatusCsr);
-        named_barrier_sync(1, 128);
+        named_barrier_sync(1, 256);
       }
 #pragma unroll
       for (int q = 0; q < 64; ++q) {
         acc[q] = -INFINITY;
         lsum[q] = 0.f;
       }
-      for (int t = 0; t < x.ntiles; ++t) {
-        int kind, ti;
-        tile_kind(x, t, kind, ti);
-        const int sb = sc & 1;
-        mbar_wait(&s_full[sb], (sc >> 1) & 1, abort_flag, p.status);
+      // ---- A1: running max of the pooled-key logits (stabiliser)
+      for (int ti = 0; ti < x.n_a1; ++ti, ++sc) {
+        if ((sc & 1) != w) continue;
+        mbar_wait(&s_full[w], my & 1, abort_flag, p.status);
         tc_fence_after();
-        const uint32_t sa = tbase + lane_addr + 64 * sb;
-        if (kind == 0) {
-          const bool valid = ti * 128 + trow < x.cand;
-          float sv[32];
-          tmem_ld32(sa, sv);
-          tc_wait_ld();
+        float sv[64];
+        tmem_ld32(s_addr, *reinterpret_cast<float(*)[32]>(&sv[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[w]);
+        ++my;
+        if (ti * 128 + trow < x.cand) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q)
-            if (valid) acc[q] = fmaxf(acc[q], sv[q]);
-          tmem_ld32(sa + 32, sv);
-          tc_wait_ld();
-          tc_fence_before();
-          mbar_arrive(&s_empty[sb]);
+          for (int q = 0; q < 64; ++q) acc[q] = fmaxf(acc[q], sv[q]);
+        }
+      }
+      // stabiliser c2 = max_J a_iJ * log2(e) + log2(64), shared by both warpgroups
+      group_reduce64<true>(acc, red, c2s, lane, gwarp, gtid);
+      if (gtid < 64) c2s[gtid] = c2s[gtid] * p.scale_log2 + 6.0f;
+      named_barrier_sync(1, 256);
 #pragma unroll
-          for (int q = 0; q < 32; ++q)
-            if (valid) acc[32 + q] = fmaxf(acc[32 + q], sv[q]);
-          ++sc;
-          if (ti == x.n_a1 - 1) {
-            // stabiliser c2 = max_J a_iJ * log2(e) + log2(64)
-            group_reduce64<true>(acc, red, c2s, lane, wq, tid);
-            if (tid < 64) c2s[tid] = c2s[tid] * p.scale_log2 + 6.0f;
-            named_barrier_sync(1, 128);
-#pragma unroll
-            for (int q = 0; q < 64; ++q) acc[q] = -c2s[q];
-          }
+      for (int q = 0; q < 64; ++q) acc[q] = -c2s[q];
+
+      // ---- A2 (unlisted pooled blocks) and E (listed blocks) tiles
+      for (int t = x.n_a1; t < x.ntiles; ++t, ++sc) {
+        if ((sc & 1) != w) continue;
+        const bool pseudo = t < x.n_a1 + x.n_a2;
+        const int ti = pseudo ? t - x.n_a1 : t - x.n_a1 - x.n_a2;
+        // which key block this thread's row belongs to (warp-uniform for E)
+        bool valid, diag = false;
+        if (pseudo) {
+          const int J = ti * 128 + trow;
+          valid = J < x.pcand && !((bitmap[J >> 5] >> (J & 31)) & 1u);
         } else {
-          bool valid, diag = false;
-          float add = 0.f;
-          if (kind == 1) {
-            const int J = ti * 128 + trow;
-            valid = J < x.pcand && !((bitmap[J >> 5] >> (J & 31)) & 1u);
-            add = 6.0f;  // weight 64 e^a on the value mean
-          } else {
-            const int idx = 2 * ti + (trow >> 6);
-            int J = -1;
-            if (idx < x.nsel) J = p.dense ? idx : __ldg(p.col_idx + x.rp + idx);
-            valid = J >= 0 && J < x.cand;
-            diag = p.causal && J == x.I;
-          }
-          const int kj = trow & 63;
-          const int pb = pc & 1;
-          uint8_t* prow = sP + pb * C::kPBytes + trow * 128;
+          const int idx = 2 * ti + (trow >> 6);
+          int J = -1;
+          if (idx < x.nsel)
+            J = p.dense ? idx : (idx < kColCache ? cols[idx] : __ldg(p.col_idx + x.rp + idx));
+          valid = J >= 0 && J < x.cand;
+          diag = p.causal && J == x.I;
+        }
+        mbar_wait(&s_full[w], my & 1, abort_flag, p.status);
+        tc_fence_after();
+        float sv[64];
+        tmem_ld32(s_addr, *reinterpret_cast<float(*)[32]>(&sv[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[w]);
+        // P^T row of this thread: 64 bf16, written as eight 16-byte chunks
+        // (128-byte swizzle: chunk c lands at c ^ (row % 8)).  The buffer is
+        // still read by this warpgroup's previous GEMM2: wait for it only
+        // after the first half of the exponentials.
+        const uint32_t pempty_par = (mp & 1) ^ 1;
+        if (!valid) {
+          mbar_wait(&g2_done[w], pempty_par, abort_flag, p.status);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(prow + ((c ^ (trow & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          const int kj = diag ? (trow & 63) : -1;  // diagonal block: key kj visible to query q iff kj <= q
+          const float wl = pseudo ? 64.f : 1.f;    // 0th-order term: weight 64 e^{a-c} on the value sum
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            float sv[32];
-            tmem_ld32(sa + 32 * h, sv);
-            tc_wait_ld();
-            if (h == 1) {
-              tc_fence_before();
-              mbar_arrive(&s_empty[sb]);
-            }
-            float pv[32];
+            uint32_t pk[16];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              const int qq = 32 * h + q;
-              float e = ex2_approx(fmaf(sv[q], p.scale_log2, acc[qq]) + add);
-              if (!valid || (diag && kj > qq)) e = 0.f;
-              lsum[qq] += e;
-              pv[q] = e;
+            for (int i = 0; i < 16; ++i) {
+              const int q0 = 32 * h + 2 * i, q1 = q0 + 1;
+              float e0 = ex2_approx(fmaf(sv[q0], p.scale_log2, acc[q0]));
+              float e1 = ex2_approx(fmaf(sv[q1], p.scale_log2, acc[q1]));
+              e0 = kj <= q0 ? e0 : 0.f;
+              e1 = kj <= q1 ? e1 : 0.f;
+              lsum[q0] = fmaf(e0, wl, lsum[q0]);
+              lsum[q1] = fmaf(e1, wl, lsum[q1]);
+              pk[i] = pack_bf16x2(e0, e1);
             }
-            if (h == 0) mbar_wait(&p_empty[pb], ((pc >> 1) & 1) ^ 1, abort_flag, p.status);
+            if (h == 0) mbar_wait(&g2_done[w], pempty_par, abort_flag, p.status);
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
               const int c = 4 * h + c4;
-              uint4 w;
-              w.x = pack_bf16x2(pv[8 * c4 + 0], pv[8 * c4 + 1]);
-              w.y = pack_bf16x2(pv[8 * c4 + 2], pv[8 * c4 + 3]);
-              w.z = pack_bf16x2(pv[8 * c4 + 4], pv[8 * c4 + 5]);
-              w.w = pack_bf16x2(pv[8 * c4 + 6], pv[8 * c4 + 7]);
-              *reinterpret_cast<uint4*>(prow + ((c ^ (trow & 7)) << 4)) = w;
+              *reinterpret_cast<uint4*>(prow + ((c ^ (trow & 7)) << 4)) =
+                  make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
             }
           }
-          fence_async_shared();
-          mbar_arrive(&p_full[pb]);
-          ++sc;
-          ++pc;
         }
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[w]);
+        ++my;
+        ++mp;
       }
 
       // ---------------------------------------------------------- epilogue
-      group_reduce64<false>(lsum, red, lsh, lane, wq, tid);
-      if (tid < 64) {
-        const float l = lsh[tid];
+      group_reduce64<false>(lsum, red, lsh, lane, gwarp, gtid);
+      if (gtid < 64) {
+        const float l = lsh[gtid];
         const bool good = l >= 0x1p-60f && l <= 0x1p60f;  // false for NaN
-        invl[tid] = good ? 1.0f / l : 0.f;
+        invl[gtid] = good ? 1.0f / l : 0.f;
         if (!good) *unit_flag = 1;
-        if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + tid] = (c2s[tid] + __log2f(l)) * kLn2;
+        if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + gtid] = (c2s[gtid] + __log2f(l)) * kLn2;
       }
-      if (tid == 0) bulk_wait_read0();  // the previous unit's store has read the staging tile
-      named_barrier_sync(1, 128);
+      if (gtid == 0) bulk_wait_read0();  // the previous unit's store has read the staging tile
+      named_barrier_sync(1, 256);
       const int ob = ul & 1;
       mbar_wait(&o_full[ob], (ul >> 1) & 1, abort_flag, p.status);
       tc_fence_after();
-      if (trow < D) {  // warp-uniform
+      if (trow < D) {  // warp-uniform; warpgroup w stores queries [32 w, 32 w + 32)
         __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sOut);
+        float ov[32];
+        tmem_ld32(tbase + lane_addr + 128 + 64 * ob + 32 * w, ov);
+        tc_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float ov[32];
-          tmem_ld32(tbase + lane_addr + 128 + 64 * ob + 32 * h, ov);
-          tc_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 32; ++q)
-            st[(32 * h + q) * D + trow] = __float2bfloat16_rn(ov[q] * invl[32 * h + q]);
-        }
+        for (int q = 0; q < 32; ++q)
+          st[(32 * w + q) * D + trow] = __float2bfloat16_rn(ov[q] * invl[32 * w + q]);
       }
       tc_fence_before();
-      mbar_arrive(&o_empty[ob]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[ob]);
       fence_async_shared();
-      named_barrier_sync(1, 128);
-      if (tid == 0) {
+      named_barrier_sync(1, 256);
+      if (gtid == 0) {
         bulk_store(p.out + static_cast<size_t>(x.row) * 64 * D, sOut, C::kOutBytes);
         bulk_commit();
         if (*unit_flag) {
@@ -585,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (tid == 0) bulk_wait0();
+    if (gtid == 0) bulk_wait0();
   }
 
   tc_fence_before();
@@ -684,7 +711,7 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
       encode_tensor_map_3d_bf16(&mk, a.k, D, a.N, bh, 64, 64) != CUDA_SUCCESS ||
       encode_tensor_map_3d_bf16(&mv, a.v, D, a.N, bh, 64, 64) != CUDA_SUCCESS ||
       encode_tensor_map_3d_bf16(&mkb, a.kbar_bf16, D, a.M, bh, 64, 64) != CUDA_SUCCESS ||
-      encode_tensor_map_3d_bf16(&mvb, a.dense ? a.kbar_bf16 : a.vbar_bf16, D, a.M, bh, 64, 64) !=
+      encode_tensor_map_3d_bf16(&mvb, a.dense ? a.kbar_bf16 : a.vsum_bf16, D, a.M, bh, 64, 64) !=
           CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   Params p;
@@ -705,6 +732,14 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  // The warpgroups re-split the registers the block was launched with
+  // (setmaxnreg); if the compiled kernel launched with fewer, the increase
+  // could never be satisfied.  Refuse to launch rather than wait forever.
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, attn_kernel<D>)) != cudaSuccess) return e;
+  if (fa.numRegs < kRegsLaunch ||
+      128 * kRegsProducer + 256 * kRegsSoftmax > kThreads * fa.numRegs)
+    return cudaErrorInvalidConfiguration;
   const int sms = device_sm_count();
   const int grid = p.units < sms ? p.units : sms;
   attn_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mkb, mvb, p);

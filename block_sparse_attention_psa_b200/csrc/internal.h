@@ -18,7 +18,7 @@ struct WorkspaceLayout {
   size_t header = 0;        // int status; int fixup_count; ... (256 B)
   size_t fixup_list = 0;    // int [B*H*M]
   size_t kbar_bf16 = 0;     // bf16 [B*H*M*d]
-  size_t vbar_bf16 = 0;     // bf16 [B*H*M*d]
+  size_t vsum_bf16 = 0;     // bf16 [B*H*M*d] (value sums)
   size_t row_count = 0;     // int [B*H*M]     (threshold routing)
   size_t row_bits = 0;      // uint32 [B*H*M*ceil(M/32)]
   size_t total = 0;
@@ -31,7 +31,7 @@ cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,
 cudaError_t launch_pool_keys_bf16(const uint16_t* k, int BH, int M, int d, uint16_t* kbar_bf16,
                                   cudaStream_t st);
 cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long n, uint16_t* kbar_bf16,
-                                 uint16_t* vbar_bf16, cudaStream_t st);
+                                 uint16_t* vsum_bf16, cudaStream_t st);
 
 // route.cu
 cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int M, int d, int k0, int causal,
@@ -46,7 +46,7 @@ struct AttnLaunch {
   const uint16_t* k;
   const uint16_t* v;
   const uint16_t* kbar_bf16;
-  const uint16_t* vbar_bf16;
+  const uint16_t* vsum_bf16;
   const float* kbar32;  // may be null in dense mode
   const float* vsum32;  // may be null in dense mode
   const int* row_ptr;   // null in dense mode

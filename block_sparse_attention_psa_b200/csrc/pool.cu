@@ -96,9 +96,8 @@ __global__ void stats_to_bf16_kernel(const float4* __restrict__ kbar, const floa
     const float4 s = vsum[i];
     kb[i] = make_uint2(f2bf(a.x) | (static_cast<uint32_t>(f2bf(a.y)) << 16),
                        f2bf(a.z) | (static_cast<uint32_t>(f2bf(a.w)) << 16));
-    const float r = 1.0f / 64.0f;
-    vb[i] = make_uint2(f2bf(s.x * r) | (static_cast<uint32_t>(f2bf(s.y * r)) << 16),
-                       f2bf(s.z * r) | (static_cast<uint32_t>(f2bf(s.w * r)) << 16));
+    vb[i] = make_uint2(f2bf(s.x) | (static_cast<uint32_t>(f2bf(s.y)) << 16),
+                       f2bf(s.z) | (static_cast<uint32_t>(f2bf(s.w)) << 16));
   }
 }
 
@@ -136,7 +135,7 @@ cudaError_t launch_pool_keys_bf16(const uint16_t* k, int BH, int M, int d, uint1
 }
 
 cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long n, uint16_t* kbar_bf16,
-                                 uint16_t* vbar_bf16, cudaStream_t st) {
+                                 uint16_t* vsum_bf16, cudaStream_t st) {
   const long long n4 = n / 4;  // n = B*H*M*d, d in {64, 128}
   long long blocks = (n4 + 255) / 256;
   const long long cap = device_sm_count() * 16LL;
@@ -144,7 +143,7 @@ cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long
   if (blocks < 1) blocks = 1;
   stats_to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
       reinterpret_cast<const float4*>(kbar), reinterpret_cast<const float4*>(vsum), n4,
-      reinterpret_cast<uint2*>(kbar_bf16), reinterpret_cast<uint2*>(vbar_bf16));
+      reinterpret_cast<uint2*>(kbar_bf16), reinterpret_cast<uint2*>(vsum_bf16));
   return cudaGetLastError();
 }
 

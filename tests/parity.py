@@ -48,6 +48,11 @@ def run_gpu(q, k, v, mode, param, causal=False, keep_first=False, want_lse=True)
                 status=status)
 
 
+def check_status(g, want=None):
+    want = psa.PSA_OK if want is None else want
+    assert g["status"] == want, f"device status {g['status']}: {psa.status_text(g['status'])}"
+
+
 def check_pool(g, q, k, v):
     qbar, kbar, vsum = O.pool(f64(q), f64(k), f64(v))
     for name, ref in (("qbar", qbar), ("kbar", kbar), ("vsum", vsum)):
@@ -109,6 +114,7 @@ def check_routing(g, s, mode, param, causal, keep_first=False):
 
 def check_output(g, q, k, v, kbar, vsum, causal, units=None):
     """Oracle fed the GPU's own block lists; compare out and lse."""
+    check_status(g)
     B, H, N, d = q.shape
     M = N // 64
     if units is None:

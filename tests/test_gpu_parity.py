@@ -56,6 +56,17 @@ def test_many_pooled_tiles():
     check_output(g, q, k, v, kbar, vsum, False, sample_units(B, H, N // 64, 40, seed=1, g=g))
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_many_units_per_cta(causal):
+    # 4 heads x 160 blocks = 640 units on 148 CTAs: units follow each other
+    # in every CTA, with 2 pooled-key tiles per unit
+    q, k, v = make_qkv(1, 4, 160 * 64, 64, "clustered", seed=14)
+    g = run_gpu(q, k, v, "topk", 0.1, causal)
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    check_routing(g, O.block_scores(qbar, kbar), "topk", 0.1, causal)
+    check_output(g, q, k, v, kbar, vsum, causal, sample_units(1, 4, 160, 60, seed=3, g=g))
+
+
 def test_single_block():
     q, k, v = make_qkv(1, 2, 64, 128, "iid", seed=6)
     for causal in (False, True):
@@ -143,6 +154,11 @@ def test_malformed_list_is_reported_not_fatal():
     lists = [np.array([0, 1])] * 7 + [np.array([3, 99])]   # J = 99 is out of range
     g = _attn_with_lists(q, k, v, lists, False)
     assert g["status"] == psa.PSA_ERR_CSR
+    # the well-formed rows are still right
+    _, kbar, vsum = O.pool(f64(q), f64(k), f64(v))
+    g_ok = dict(g, status=psa.PSA_OK)
+    g_ok["row_ptr"], g_ok["col_idx"] = O._to_csr(lists[:7] + [np.array([3])])
+    check_output(g_ok, q, k, v, kbar, vsum, False, [(0, 0, I) for I in range(7)])
     # the device is still healthy afterwards
     g2 = _attn_with_lists(q, k, v, [np.array([0, 1])] * 8, False)
     assert g2["status"] == psa.PSA_OK
