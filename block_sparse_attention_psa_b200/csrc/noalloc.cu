@@ -1,0 +1,126 @@
+// noalloc.cu -- psa_attn_noalloc: the attention step without a caller
+// workspace, for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc (or any allocating routine) at the
+// point where they run attention: plugins inside frameworks whose device
+// memory all comes from the framework's own pool, or real-time and
+// safety-critical loops that forbid allocation after start-up.  This entry point needs nothing from them but
+// the inputs and outputs: its scratch (the bf16 copies of the pooled keys
+// and value sums, the status word and the fixup list) lives in one
+// file-scope device array below.
+//
+// That array is shared by every call on a device and keeps the previous
+// call's contents; the parts that must start at zero (status word, fixup
+// counter) are cleared by each call.  Two calls whose kernels overlap on the
+// GPU (different streams, no ordering between them) therefore race on it.
+#include <climits>
+#include <mutex>
+
+#include "internal.h"
+#include "psa.h"
+
+namespace {
+
+// 16 MiB of scratch, 256-byte aligned.  Every GPU that loads this library
+// holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Scratch bytes the attention step needs: header, fixup list, bf16 pooled keys
+// and bf16 value sums (the same layout as the front of the workspace).
+size_t scratch_bytes(long long BH, long long M, long long d) {
+  return 256 + align256(static_cast<size_t>(BH * M) * 4) + 2 * align256(static_cast<size_t>(BH * M * d) * 2);
+}
+
+// Device address of the scratch array on the current device.  The host-side
+// symbol is only a stand-in, never a device address: it is looked up once
+// per device, with that device current, and cached.
+int scratch_for_current_device(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PSA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return PSA_ERR_CUDA;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return PSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar,
+                     const float* vsum, const int* row_ptr, const int* col_idx, size_t col_capacity, int B, int H,
+                     int N, int d, int block_size, int causal, psa_bf16_t* out, float* lse, int* status,
+                     void* stream) {
+  if (!q || !k || !v || !kbar || !vsum || !row_ptr || !col_idx || !out) return PSA_ERR_ARG;
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return PSA_ERR_ARG;
+  if (block_size != psa::kBlock || (d != 64 && d != 128)) return PSA_ERR_UNSUPPORTED;
+  if (N % psa::kBlock) return PSA_ERR_SHAPE;
+  if (N / psa::kBlock > psa::kMaxBlocks) return PSA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N * d >= (1LL << 31)) return PSA_ERR_SHAPE;
+  if (causal != 0 && causal != 1) return PSA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kbar) ||
+      !aligned16(vsum) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+      (status && (reinterpret_cast<uintptr_t>(status) & 3u)))
+    return PSA_ERR_ARG;
+  const long long bh = static_cast<long long>(B) * H;
+  const int M = N / psa::kBlock;
+  if (scratch_bytes(bh, M, d) > kNoAllocScratchBytes) return PSA_ERR_CAPACITY;  // shape too large
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10)
+    return PSA_ERR_DEVICE;
+  void* base = nullptr;
+  int s = scratch_for_current_device(&base);
+  if (s != PSA_OK) return s;
+  char* ws = static_cast<char*>(base);
+  const size_t off_fix = 256;
+  const size_t off_kb = off_fix + align256(static_cast<size_t>(bh * M) * 4);
+  const size_t off_vs = off_kb + align256(static_cast<size_t>(bh * M * d) * 2);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the status word and the fixup counter must start at zero on every call
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
+  uint16_t* kb16 = reinterpret_cast<uint16_t*>(ws + off_kb);
+  uint16_t* vs16 = reinterpret_cast<uint16_t*>(ws + off_vs);
+  if (psa::launch_stats_to_bf16(kbar, vsum, bh * M * d, kb16, vs16, st) != cudaSuccess) return PSA_ERR_CUDA;
+  psa::AttnLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.kbar_bf16 = kb16;
+  a.vsum_bf16 = vs16;
+  a.kbar32 = kbar;
+  a.vsum32 = vsum;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.col_cap = col_capacity > static_cast<size_t>(LLONG_MAX) ? LLONG_MAX : static_cast<long long>(col_capacity);
+  a.out = out;
+  a.lse = lse;
+  a.BH = static_cast<int>(bh);
+  a.N = N;
+  a.M = M;
+  a.d = d;
+  a.causal = causal;
+  a.dense = 0;
+  a.status = reinterpret_cast<int*>(ws);
+  a.fixup_count = reinterpret_cast<int*>(ws) + 1;
+  a.fixup_list = reinterpret_cast<int*>(ws + off_fix);
+  if (psa::launch_attn(a, st) != cudaSuccess) return PSA_ERR_CUDA;
+  if (status && cudaMemcpyAsync(status, ws, sizeof(int), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return PSA_ERR_CUDA;
+  return PSA_OK;
+}
+
+}  // extern "C"

@@ -29,7 +29,8 @@ PSA_ERR_CSR = 7
 PSA_ERR_DEVICE = 8
 
 EXPORTS = ("psa_status_string", "psa_version", "psa_workspace_size", "psa_route_capacity", "psa_pool",
-           "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense", "psa_read_status")
+           "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense", "psa_read_status",
+           "psa_attn_noalloc")
 
 _lib = None
 
@@ -53,6 +54,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "psa_attn": (I, [P, P, P, P, P, P, P, Z, I, I, I, I, I, I, P, P, P, Z, P]),
         "psa_dense": (I, [P, P, P, I, I, I, I, I, P, P, P, Z, P]),
         "psa_read_status": (I, [P, ctypes.POINTER(I), P]),
+        "psa_attn_noalloc": (I, [P, P, P, P, P, P, P, Z, I, I, I, I, I, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -195,6 +197,22 @@ def psa_dense(q, k, v, causal: bool = False, ws=None, out=None, lse=None, want_l
         _ptr(q), _ptr(k), _ptr(v), B, H, N, d, int(causal), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
         _stream(stream)))
     return (out, lse) if lse is not None else out
+
+
+def psa_attn_noalloc(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_size: int = 64,
+                     out=None, lse=None, status=None, stream=None):
+    """psa_attn without a workspace, for callers that cannot allocate device
+    memory (framework plugins restricted to the framework's own pool, loops
+    that forbid allocation after start-up): the library's own 16 MiB scratch
+    array is used instead, and calls that overlap on the GPU race on it.  ``status`` is an optional device
+    int32 tensor that receives this call's device status word."""
+    B, H, N, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check("psa_attn_noalloc", lib().psa_attn_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+        B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(status), _stream(stream)))
+    return out
 
 
 def psa_read_status(ws, stream=None) -> int:

@@ -173,6 +173,26 @@ PSA_API int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t
               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Attention without a workspace, for callers that cannot allocate device
+ * memory (the method's sources have no counterpart: this is an interface
+ * choice).  Same computation, arguments and errors as psa_attn, minus the
+ * workspace: the scratch (bf16 pooled keys and value sums, status word,
+ * fixup list) lives in a 16 MiB array inside the library, so shapes need
+ * 256 + 4*B*H*M + 4*B*H*M*d bytes (each part rounded up to 256 bytes) to fit
+ * in 16 MiB, else PSA_ERR_CAPACITY.  The first call on a device looks up the
+ * array's device address (make it before any stream capture).  Every call on
+ * a device shares the array: calls whose work overlaps on the GPU race.
+ * `status` (device int, nullable) receives the device status word of this
+ * call (PSA_OK, PSA_ERR_CSR or PSA_ERR_TIMEOUT) in stream order.  Never
+ * allocates device memory.
+ */
+PSA_API int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v,
+                             const float* kbar, const float* vsum,
+                             const int* row_ptr, const int* col_idx, size_t col_capacity,
+                             int B, int H, int N, int d, int block_size, int causal,
+                             psa_bf16_t* out, float* lse, int* status, void* stream);
+
+/*
  * Synchronises `stream`, then copies the device status word of `workspace`
  * into *status (host pointer): PSA_OK, or the first device-side error
  * recorded since the last call that reset it (psa_route_thresh, psa_attn
