@@ -323,7 +323,7 @@ def gpu_arm(args):
                    "l2": "flushed between steps (512 MB write outside the timed events)"},
         "roofline": {"bound": "tensor", "kernel": "attn_kernel (psa_attn call)",
                      "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / tc_peak, 4), "traffic": None,
+                     "frac": round(achieved / tc_peak, 4), "traffic": recorded_traffic(st.name),
                      "peak_source": peaks["source"] + " bf16 burst"},
         "kernels": {"pool_ms": round(pool_avg, 4), "route_ms": round(route_avg, 4), "attn_ms": round(attn_avg, 4),
                     "pool_gbs": round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3) / 1e9, 1),
@@ -348,6 +348,27 @@ def gpu_arm(args):
         import torch.distributed as dist
 
         dist.destroy_process_group()
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary of this
+    workload, if the kernel source still matches the one that was captured
+    (else None: the counters no longer describe the kernel)."""
+    import hashlib
+    import re
+
+    prof = os.path.join(ROOT, "profiles", f"attn_kernel_{workload}.md")
+    src = os.path.join(ROOT, "block_sparse_attention_psa_b200", "csrc", "attn.cu")
+    try:
+        text = open(prof).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    m_sha = re.search(r"attn.cu sha256 prefix at capture: ([0-9a-f]{16})", text)
+    m_tr = re.search(r"traffic_bytes_per_launch: (\d+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != sha:
+        return None
+    return int(m_tr.group(1))
 
 
 def _peaks():
