@@ -157,7 +157,8 @@ class Step:
         self.stats = tuple(torch.empty(B, H, M, d, **f32) for _ in range(3))
         cap = psa.psa_route_capacity(B, H, M, self.causal)
         i32 = dict(dtype=torch.int32, device=device)
-        self.csr = (torch.empty(B * H * M + 1, **i32), torch.empty(cap, **i32), torch.empty(1, **i32))
+        self.csr = (torch.empty(B * H * M + 1, **i32), torch.empty(cap, **i32), torch.empty(1, **i32),
+                    torch.empty(B * H * M, dtype=torch.float32, device=device))
         self.ws = psa.workspace(B, H, self.N, d, device)
         self.out = torch.empty_like(self.q)
         self.out_host = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
@@ -182,7 +183,7 @@ class Step:
         if ev:
             ev[2].record(s)
         psa.psa_attn(self.q, self.k, self.v, kbar, vsum, self.csr[0], self.csr[1], self.causal, ws=self.ws,
-                     out=self.out, stream=s)
+                     out=self.out, row_max=self.csr[3], stream=s)
         if ev:
             ev[3].record(s)
 

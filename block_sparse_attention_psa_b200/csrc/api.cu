@@ -147,8 +147,9 @@ int psa_pool(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int 
 }
 
 int psa_route_topk(const float* qbar, const float* kbar, int B, int H, int M, int d, float density, int causal,
-                   int* row_ptr, int* col_idx, size_t capacity, int* nnz_out, void* stream) {
+                   int* row_ptr, int* col_idx, size_t capacity, int* nnz_out, float* row_max, void* stream) {
   if (!qbar || !kbar || !row_ptr || !col_idx || !nnz_out) return PSA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(row_max) & 3u) return PSA_ERR_ARG;
   if (M <= 0) return PSA_ERR_ARG;
   if (M > kMaxBlocks) return PSA_ERR_UNSUPPORTED;
   int s = check_shape(B, H, M * kBlock, d, kBlock);
@@ -165,14 +166,15 @@ int psa_route_topk(const float* qbar, const float* kbar, int B, int H, int M, in
   if (total > INT_MAX || static_cast<size_t>(total) > capacity) return PSA_ERR_CAPACITY;
   if ((s = check_device()) != PSA_OK) return s;
   return cuda_status(psa::launch_route_topk(qbar, kbar, static_cast<int>(bh), M, d, static_cast<int>(k0),
-                                            causal, row_ptr, col_idx, total, nnz_out,
+                                            causal, row_ptr, col_idx, total, nnz_out, row_max,
                                             static_cast<cudaStream_t>(stream)));
 }
 
 int psa_route_thresh(const float* qbar, const float* kbar, int B, int H, int M, int d, float alpha, int causal,
-                     int keep_first, int* row_ptr, int* col_idx, size_t capacity, int* nnz_out, void* workspace,
-                     size_t workspace_bytes, void* stream) {
+                     int keep_first, int* row_ptr, int* col_idx, size_t capacity, int* nnz_out, float* row_max,
+                     void* workspace, size_t workspace_bytes, void* stream) {
   if (!qbar || !kbar || !row_ptr || !col_idx || !nnz_out || !workspace) return PSA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(row_max) & 3u) return PSA_ERR_ARG;
   if (M <= 0) return PSA_ERR_ARG;
   if (M > kMaxBlocks) return PSA_ERR_UNSUPPORTED;
   int s = check_shape(B, H, M * kBlock, d, kBlock);
@@ -189,21 +191,21 @@ int psa_route_thresh(const float* qbar, const float* kbar, int B, int H, int M, 
   return cuda_status(psa::launch_route_thresh(qbar, kbar, static_cast<int>(bh), M, d, alpha, causal, keep_first,
                                               row_ptr, col_idx, cap, nnz_out,
                                               reinterpret_cast<int*>(ws + L.row_count),
-                                              reinterpret_cast<uint32_t*>(ws + L.row_bits),
+                                              reinterpret_cast<uint32_t*>(ws + L.row_bits), row_max,
                                               static_cast<cudaStream_t>(stream)));
 }
 
 int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar, const float* vsum,
-             const int* row_ptr, const int* col_idx, size_t col_capacity, int B, int H, int N, int d,
-             int block_size, int causal, psa_bf16_t* out, float* lse, void* workspace, size_t workspace_bytes,
-             void* stream) {
+             const int* row_ptr, const int* col_idx, size_t col_capacity, const float* row_max, int B, int H,
+             int N, int d, int block_size, int causal, psa_bf16_t* out, float* lse, void* workspace,
+             size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !kbar || !vsum || !row_ptr || !col_idx || !out || !workspace) return PSA_ERR_ARG;
   int s = check_shape(B, H, N, d, block_size);
   if (s != PSA_OK) return s;
   if (causal != 0 && causal != 1) return PSA_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kbar) ||
       !aligned16(vsum) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (reinterpret_cast<uintptr_t>(row_max) & 3u))
     return PSA_ERR_ARG;
   const long long bh = static_cast<long long>(B) * H;
   const int M = N / kBlock;
@@ -229,6 +231,7 @@ int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, cons
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
   a.col_cap = col_capacity > static_cast<size_t>(LLONG_MAX) ? LLONG_MAX : static_cast<long long>(col_capacity);
+  a.row_max = row_max;
   a.out = out;
   a.lse = lse;
   a.BH = static_cast<int>(bh);

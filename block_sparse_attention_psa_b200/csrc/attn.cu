@@ -18,19 +18,24 @@
 //       O^T[d x 64 queries]        += V_tile^T . P^T   (A = V, MN-major;
 //                                      B = P^T, MN-major)
 //    with S^T and O^T in TMEM (tcgen05.mma, f32 accumulate).
-//  * Softmax stabiliser: the per-query constant c_i = max_J (a_iJ + ln 64)
-//    over all candidate blocks, a_iJ = q_i.kbar_J/sqrt(d), taken in a first
-//    sweep over the pooled keys.  Because the mean of a block's logits is
-//    a_iJ, the largest term of the row is >= e^{c_i - ln 64}; every term
-//    relative to c_i stays in fp32 range unless one key's logit exceeds its
-//    block mean by ~90.  Rows whose final sum leaves [2^-60, 2^60] are
-//    recomputed exactly by a fixup kernel.  With a fixed stabiliser the
-//    running output never needs rescaling, so there is no correction step.
-//  * Tile stream of a unit: A1 tiles (pooled keys, for c), A2 tiles (pooled
-//    keys + pooled values of the unlisted blocks), E tiles (two listed key
-//    blocks each).  Warp 0: TMA producer.  Warp 1: tcgen05 issuer (one
-//    thread) and TMEM owner.  Warps 2-5: softmax + epilogue, one thread per
-//    TMEM lane (= key row of S^T, = feature row of O^T).
+//  * Softmax stabiliser: one constant per query block, in log2 units
+//    c2 = max_J s_IJ * log2(e) + log2(64), s_IJ = qbar_I.kbar_J/sqrt(d) over
+//    the candidate blocks: the router's row maximum when it is passed in,
+//    else computed here from q and the pooled keys.  It approximates the
+//    largest 0th-order exponent of the block's queries; each query's terms
+//    stay in fp32 range unless its logits sit ~90 (natural units) away from
+//    it.  Rows whose final sum leaves [2^-60, 2^60] are recomputed exactly by
+//    a fixup kernel.  With a fixed stabiliser the running output never needs
+//    rescaling, so there is no correction step.
+//  * Tile stream of a unit: A2 tiles (128 pooled keys + pooled value sums
+//    of the unlisted blocks) then E tiles (two listed key blocks each).
+//    Warp group 0: warp 0 loads Q and K tiles, warp 2 loads V tiles (TMA);
+//    warp 1 issues S^T = K.Q^T and owns TMEM, warp 3 issues O^T += V^T.P^T
+//    (one thread each).  Warp groups 1 and 2 take alternate tiles for the
+//    softmax, one thread per TMEM lane (= key row of S^T), and share the
+//    epilogue (one thread per feature row of O^T).  Two S^T buffers and two
+//    O^T accumulators (by unit parity) let consecutive tiles and units
+//    overlap.
 //  * Every wait is bounded; on a timeout all roles stop, drain what is in
 //    flight, free TMEM and return with PSA_ERR_TIMEOUT recorded.
 #include <cuda_bf16.h>
@@ -42,8 +47,8 @@ namespace psa {
 namespace {
 
 constexpr int kThreads = 384;     // WG0: TMA producers (warps 0, 2), MMA issuers (warps 1, 3); WG1, WG2: softmax
-constexpr int kRegsProducer = 56;  // setmaxnreg split: 128 x 56 + 256 x 224 = 384 x 168
-constexpr int kRegsSoftmax = 224;
+constexpr int kRegsProducer = 72;  // setmaxnreg split: 128 x 72 + 256 x 216 = 384 x 168
+constexpr int kRegsSoftmax = 216;
 constexpr int kRegsLaunch = 168;
 constexpr int kColCache = 1024;   // listed blocks of a unit kept in shared memory
 constexpr float kLn2 = 0.6931471805599453f;
@@ -62,9 +67,10 @@ struct Cfg {
   static constexpr int kOffP = kOffV + kNV * kKVBytes;   // one P^T tile per softmax warpgroup
   static constexpr int kOffOut = kOffP + 2 * kPBytes;
   static constexpr int kOffMisc = kOffOut + kOutBytes;
-  // misc: 32 barriers (256 B) + tmem slot / flags (256 B) + red[8][64] f32 +
-  // c2[64] + invl[64] + l[64] + bitmap[kMaxBlocks / 32] + cols[kColCache]
-  static constexpr int kMiscBytes = 256 + 256 + 8 * 64 * 4 + 3 * 64 * 4 + kMaxBlocks / 8 + kColCache * 4;
+  // misc: 32 barriers (256 B) + tmem slot / flags (256 B) + red[8][128 + 1]
+  // f32 + qbar[128] + invl[64] + l[64] + bitmap[kMaxBlocks / 32] + cols[kColCache]
+  static constexpr int kMiscBytes = 256 + 256 + (8 * 128 + 8) * 4 + 128 * 4 + 2 * 64 * 4 + kMaxBlocks / 8 +
+                                    kColCache * 4;
   static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
   // kind::f16, bf16 x bf16 -> f32.  GEMM1: M=128 keys, N=64 queries, both
   // K-major.  GEMM2: M=128 (feature rows), N=64 queries, both MN-major.
@@ -73,9 +79,12 @@ struct Cfg {
 };
 
 struct Params {
+  const uint16_t* q;          // bf16 [BH, N, D]: block means for the stabiliser
+  const uint16_t* kbar16;     // bf16 [BH, M, D]: pooled keys
   const int* row_ptr;
   const int* col_idx;
   long long col_cap;
+  const float* row_max;       // per row max block score s_IJ (nullable)
   __nv_bfloat16* out;
   float* lse;
   int BH, M, causal, dense, units;
@@ -87,7 +96,7 @@ struct Params {
 
 // Everything every role needs to agree on about one work unit.
 struct Unit {
-  int bh, I, row, rp, nsel, cand, pcand, n_a1, n_a2, n_e, ntiles;
+  int bh, I, row, rp, nsel, cand, pcand, n_a2, n_e, ntiles;
   bool bad;  // row_ptr entries out of range
 };
 
@@ -115,28 +124,21 @@ __device__ __forceinline__ Unit make_unit(int u, const Params& p) {
       x.nsel = b - a;
     }
   }
-  x.n_a1 = (x.cand + 127) / 128;
   const bool a2 = !p.dense && x.pcand > 0 && x.nsel < x.cand;
   x.n_a2 = a2 ? (x.pcand + 127) / 128 : 0;
   int ne = (x.nsel + 1) / 2;
   if (ne == 0 && x.n_a2 == 0) ne = 1;  // keep one product so O is defined
   x.n_e = ne;
-  x.ntiles = x.n_a1 + x.n_a2 + x.n_e;
+  x.ntiles = x.n_a2 + x.n_e;
   return x;
 }
 
-// tile t of a unit -> kind (0 = A1, 1 = A2, 2 = E) and index within the kind
-__device__ __forceinline__ void tile_kind(const Unit& x, int t, int& kind, int& ti) {
-  if (t < x.n_a1) {
-    kind = 0;
-    ti = t;
-  } else if (t < x.n_a1 + x.n_a2) {
-    kind = 1;
-    ti = t - x.n_a1;
-  } else {
-    kind = 2;
-    ti = t - x.n_a1 - x.n_a2;
-  }
+// tile t of a unit: pooled (A2, unlisted blocks) or exact (E, listed
+// blocks), and its index within its kind
+__device__ __forceinline__ bool tile_is_pooled(const Unit& x, int t, int& ti) {
+  const bool pooled = t < x.n_a2;
+  ti = pooled ? t : t - x.n_a2;
+  return pooled;
 }
 
 // Bounded wait that ignores the abort flag (teardown only).
@@ -190,6 +192,68 @@ __device__ __forceinline__ void reg_alloc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
 }
 
+// Exponentials of one half (32 queries) of this thread's S^T row, packed to
+// bf16 pairs, with the denominator shares accumulated.  kMode 0: listed
+// block; 1: pooled key of an unlisted block (weight 64 e^{a-c}, masked by
+// `keep`); 2: diagonal block under the causal mask (key kj visible to query
+// q iff kj <= q).
+// Query pairs (bit i = queries 2i, 2i+1 of a half) whose exponentials are
+// computed on the FMA pipe instead of the special-function unit.
+#ifndef PSA_POLY_PAIRS
+#define PSA_POLY_PAIRS 0x0u
+#endif
+// Packed fp32 pair instructions for the scale/bias and the denominators.
+#ifndef PSA_F32X2
+#define PSA_F32X2 1
+#endif
+constexpr uint32_t kPolyPairs = PSA_POLY_PAIRS;
+
+template <int kMode, int kHalf>
+__device__ __forceinline__ void exp_half(const float (&sv)[64], float bias, float (&lsum)[64], float sl, int kj,
+                                         bool keep, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int q0 = 32 * kHalf + 2 * i, q1 = q0 + 1;
+    float x0, x1;
+#if PSA_F32X2
+    ffma2(x0, x1, sv[q0], sv[q1], sl, sl, bias, bias);
+#else
+    x0 = fmaf(sv[q0], sl, bias);
+    x1 = fmaf(sv[q1], sl, bias);
+#endif
+    float e0, e1;
+    if ((kPolyPairs >> i) & 1u) {
+      e0 = exp2_poly(x0);
+      e1 = exp2_poly(x1);
+    } else {
+      e0 = ex2_approx(x0);
+      e1 = ex2_approx(x1);
+    }
+    if (kMode == 1) {
+      e0 = keep ? e0 : 0.f;
+      e1 = keep ? e1 : 0.f;
+#if PSA_F32X2
+      ffma2(lsum[q0], lsum[q1], e0, e1, 64.f, 64.f, lsum[q0], lsum[q1]);
+#else
+      lsum[q0] = fmaf(e0, 64.f, lsum[q0]);
+      lsum[q1] = fmaf(e1, 64.f, lsum[q1]);
+#endif
+    } else {
+      if (kMode == 2) {
+        e0 = kj <= q0 ? e0 : 0.f;
+        e1 = kj <= q1 ? e1 : 0.f;
+      }
+#if PSA_F32X2
+      fadd2(lsum[q0], lsum[q1], lsum[q0], lsum[q1], e0, e1);
+#else
+      lsum[q0] += e0;
+      lsum[q1] += e1;
+#endif
+    }
+    pk[i] = pack_bf16x2(e0, e1);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -221,9 +285,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* unit_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   volatile int* stop_s = reinterpret_cast<volatile int*>(tmem_slot + 3);
-  float* red = reinterpret_cast<float*>(smem + C::kOffMisc + 512);
-  float* c2s = red + 8 * 64;
-  float* invl = c2s + 64;
+  float* red = reinterpret_cast<float*>(smem + C::kOffMisc + 512);  // [8][128] + [8]
+  float* qbs = red + 8 * 128 + 8;  // block mean of the unit's queries [128]
+  float* invl = qbs + 128;
   float* lsh = invl + 64;
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(lsh + 64);
   int* cols = reinterpret_cast<int*>(bitmap + kMaxBlocks / 32);
@@ -293,12 +357,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       int colv = 0;
       for (int t = 0; t < x.ntiles && ok; ++t, ++sc) {
-        int kind, ti;
-        tile_kind(x, t, kind, ti);
-        if (!keys && kind == 0) continue;  // pooled-key max tiles have no value operand
+        int ti;
+        const bool pooled = tile_is_pooled(x, t, ti);
         int y0, y1;
         const CUtensorMap* m;
-        if (kind == 2) {
+        if (!pooled) {
           m = keys ? &tmK : &tmV;
           const int e2 = 2 * ti;
           int j1, j2;
@@ -402,7 +465,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ul) {
         const Unit x = make_unit(u, p);
         const int ob = ul & 1;
-        sc += x.n_a1;
         const int g2_total = x.n_a2 + x.n_e;
         for (int g = 0; g < g2_total; ++g, ++sc) {
           const int pb = sc & 1;
@@ -438,13 +500,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gwarp = gtid >> 5;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t s_addr = tbase + lane_addr + 64 * w;
-    uint8_t* prow = sP + w * C::kPBytes + trow * 128;
-    float acc[64];   // running max in A1, then minus the stabiliser (log2 units)
+    const uint32_t prow = smem_u32(sP + w * C::kPBytes) + trow * 128;  // this thread's P^T row
     float lsum[64];  // this thread's share of the denominators
     // Waits in this group never leave the control flow: after a timeout
     // (abort raised) they return at once and the group runs on with garbage
     // data until the next unit boundary, where all 256 threads take the same
     // stop decision.  This keeps every named barrier matched.
+    // turn-taking for the exponentials: warpgroup 0 owns tile 0, so it starts
+    if (w == 1) named_barrier_arrive(2, 256);
+    float c2 = 0.f;  // stabiliser of the current unit (log2 units)
     int sc = 0;   // running tile index (both warpgroups count every tile)
     int my = 0;   // tiles of this warpgroup so far (S buffer phase)
     int mp = 0;   // P^T tiles written by this warpgroup so far (P buffer phase)
@@ -475,40 +539,81 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_barrier_sync(1, 256);
       }
 #pragma unroll
-      for (int q = 0; q < 64; ++q) {
-        acc[q] = -INFINITY;
-        lsum[q] = 0.f;
-      }
-      // ---- A1: running max of the pooled-key logits (stabiliser)
-      for (int ti = 0; ti < x.n_a1; ++ti, ++sc) {
-        if ((sc & 1) != w) continue;
-        mbar_wait(&s_full[w], my & 1, abort_flag, p.status);
-        tc_fence_after();
-        float sv[64];
-        tmem_ld32(s_addr, *reinterpret_cast<float(*)[32]>(&sv[0]));
-        tmem_ld32(s_addr + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
-        tc_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[w]);
-        ++my;
-        if (ti * 128 + trow < x.cand) {
+      for (int q = 0; q < 64; ++q) lsum[q] = 0.f;
+      // Stabiliser of the whole query block (log2 units): c2 = max over the
+      // candidate blocks of qbar_I . kbar_J / sqrt(d) * log2(e) + log2(64),
+      // with qbar_I the mean of the block's queries.  Any constant within a
+      // few tens of the rows' largest logits keeps every term in range; rows
+      // whose sum still leaves [2^-60, 2^60] are recomputed by the fixup.
+      if (p.row_max) {
+        // the router's largest block score of this row, qbar_I . kbar_J / sqrt(d)
+        c2 = __ldg(p.row_max + x.row) * 1.4426950408889634f + 6.0f;
+      } else {
+        constexpr int kCh = D / 8;             // 16-byte chunks of a row
+        constexpr int kGr = 256 / kCh;         // row groups
+        const int ch = gtid % kCh, gr = gtid / kCh;
+        const uint4* qrow = reinterpret_cast<const uint4*>(p.q) + (static_cast<size_t>(x.row) * 64) * kCh + ch;
+        float part[8];
 #pragma unroll
-          for (int q = 0; q < 64; ++q) acc[q] = fmaxf(acc[q], sv[q]);
+        for (int i = 0; i < 8; ++i) part[i] = 0.f;
+#pragma unroll
+        for (int r = gr; r < 64; r += kGr) {
+          const uint4 w4 = __ldg(qrow + static_cast<size_t>(r) * kCh);
+          const uint32_t u[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            part[2 * i] += __uint_as_float(u[i] << 16);
+            part[2 * i + 1] += __uint_as_float(u[i] & 0xffff0000u);
+          }
         }
-      }
-      // stabiliser c2 = max_J a_iJ * log2(e) + log2(64), shared by both warpgroups
-      group_reduce64<true>(acc, red, c2s, lane, gwarp, gtid);
-      if (gtid < 64) c2s[gtid] = c2s[gtid] * p.scale_log2 + 6.0f;
-      named_barrier_sync(1, 256);
 #pragma unroll
-      for (int q = 0; q < 64; ++q) acc[q] = -c2s[q];
+        for (int o = kCh; o < 32; o <<= 1)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
+        if (lane < kCh) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) red[gwarp * 64 * 2 + ch * 8 + i] = part[i];  // [8 warps][<=128]
+        }
+        named_barrier_sync(1, 256);
+        if (gtid < D) {
+          float sum = 0.f;
+#pragma unroll
+          for (int wv = 0; wv < 8; ++wv) sum += red[wv * 128 + gtid];
+          qbs[gtid] = sum * (1.0f / 64.0f);
+        }
+        named_barrier_sync(1, 256);
+        float mx = -INFINITY;
+        const uint4* kb = reinterpret_cast<const uint4*>(p.kbar16) + static_cast<size_t>(x.bh) * p.M * kCh;
+        for (int J = gtid; J < x.cand; J += 256) {
+          float dot = 0.f;
+#pragma unroll 4
+          for (int c = 0; c < kCh; ++c) {
+            const uint4 w4 = __ldg(kb + static_cast<size_t>(J) * kCh + c);
+            const uint32_t u[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dot = fmaf(qbs[8 * c + 2 * i], __uint_as_float(u[i] << 16), dot);
+              dot = fmaf(qbs[8 * c + 2 * i + 1], __uint_as_float(u[i] & 0xffff0000u), dot);
+            }
+          }
+          mx = fmaxf(mx, dot);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) red[1024 + gwarp] = mx;
+        named_barrier_sync(1, 256);
+        float m8 = red[1024];
+#pragma unroll
+        for (int wv = 1; wv < 8; ++wv) m8 = fmaxf(m8, red[1024 + wv]);
+        c2 = m8 * p.scale_log2 + 6.0f;
+      }
+      const float bias = -c2;
 
       // ---- A2 (unlisted pooled blocks) and E (listed blocks) tiles
-      for (int t = x.n_a1; t < x.ntiles; ++t, ++sc) {
+      for (int t = 0; t < x.ntiles; ++t, ++sc) {
         if ((sc & 1) != w) continue;
-        const bool pseudo = t < x.n_a1 + x.n_a2;
-        const int ti = pseudo ? t - x.n_a1 : t - x.n_a1 - x.n_a2;
+        int ti;
+        const bool pseudo = tile_is_pooled(x, t, ti);
         // which key block this thread's row belongs to (warp-uniform for E)
         bool valid, diag = false;
         if (pseudo) {
@@ -532,41 +637,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[w]);
         // P^T row of this thread: 64 bf16, written as eight 16-byte chunks
-        // (128-byte swizzle: chunk c lands at c ^ (row % 8)).  The buffer is
-        // still read by this warpgroup's previous GEMM2: wait for it only
-        // after the first half of the exponentials.
-        const uint32_t pempty_par = (mp & 1) ^ 1;
-        if (!valid) {
-          mbar_wait(&g2_done[w], pempty_par, abort_flag, p.status);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(prow + ((c ^ (trow & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        // 0 listed block, 1 pooled key, 2 causal diagonal, 3 nothing (zero row);
+        // warp-uniform except the pooled-key validity, which is a select
+        const int mode = pseudo ? 1 : (!valid ? 3 : (diag ? 2 : 0));
+        const int kj = trow & 63;
+        // The two warpgroups share the special-function units: they take
+        // turns (tile parity order) for the exponentials, so one warpgroup's
+        // exponentials overlap the other's loads, stores and waits.
+        named_barrier_sync(2 + w, 256);
+        uint32_t pk[32];
+        if (mode == 0) {
+          exp_half<0, 0>(sv, bias, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+          exp_half<0, 1>(sv, bias, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+        } else if (mode == 1) {
+          exp_half<1, 0>(sv, bias, lsum, p.scale_log2, kj, valid, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+          exp_half<1, 1>(sv, bias, lsum, p.scale_log2, kj, valid, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+        } else if (mode == 2) {
+          exp_half<2, 0>(sv, bias, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+          exp_half<2, 1>(sv, bias, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
         } else {
-          const int kj = diag ? (trow & 63) : -1;  // diagonal block: key kj visible to query q iff kj <= q
-          const float wl = pseudo ? 64.f : 1.f;    // 0th-order term: weight 64 e^{a-c} on the value sum
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int q0 = 32 * h + 2 * i, q1 = q0 + 1;
-              float e0 = ex2_approx(fmaf(sv[q0], p.scale_log2, acc[q0]));
-              float e1 = ex2_approx(fmaf(sv[q1], p.scale_log2, acc[q1]));
-              e0 = kj <= q0 ? e0 : 0.f;
-              e1 = kj <= q1 ? e1 : 0.f;
-              lsum[q0] = fmaf(e0, wl, lsum[q0]);
-              lsum[q1] = fmaf(e1, wl, lsum[q1]);
-              pk[i] = pack_bf16x2(e0, e1);
-            }
-            if (h == 0) mbar_wait(&g2_done[w], pempty_par, abort_flag, p.status);
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const int c = 4 * h + c4;
-              *reinterpret_cast<uint4*>(prow + ((c ^ (trow & 7)) << 4)) =
-                  make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
-            }
-          }
+          for (int i = 0; i < 32; ++i) pk[i] = 0u;
         }
+        named_barrier_arrive(2 + (w ^ 1), 256);
+        // P^T row of this thread: 64 bf16 as eight 16-byte chunks (128-byte
+        // swizzle: chunk c lands at c ^ (row % 8)), once this warpgroup's
+        // previous GEMM2 has finished reading the buffer
+        mbar_wait(&g2_done[w], (mp & 1) ^ 1, abort_flag, p.status);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(prow + ((c ^ (trow & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         fence_async_shared();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[w]);
@@ -581,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool good = l >= 0x1p-60f && l <= 0x1p60f;  // false for NaN
         invl[gtid] = good ? 1.0f / l : 0.f;
         if (!good) *unit_flag = 1;
-        if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + gtid] = (c2s[gtid] + __log2f(l)) * kLn2;
+        if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + gtid] = (c2 + __log2f(l)) * kLn2;
       }
       if (gtid == 0) bulk_wait_read0();  // the previous unit's store has read the staging tile
       named_barrier_sync(1, 256);
@@ -612,6 +712,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    // the last tile's owner handed the turn to the other warpgroup: take it
+    if ((sc & 1) == w) named_barrier_sync(2 + w, 256);
     if (gtid == 0) bulk_wait0();
   }
 
@@ -715,9 +817,12 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
           CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   Params p;
+  p.q = a.q;
+  p.kbar16 = a.kbar_bf16;
   p.row_ptr = a.row_ptr;
   p.col_idx = a.col_idx;
   p.col_cap = a.col_cap;
+  p.row_max = a.row_max;
   p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
   p.BH = a.BH;

@@ -35,10 +35,12 @@ cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long
 
 // route.cu
 cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int M, int d, int k0, int causal,
-                              int* row_ptr, int* col_idx, long long total, int* nnz_out, cudaStream_t st);
+                              int* row_ptr, int* col_idx, long long total, int* nnz_out, float* row_max,
+                              cudaStream_t st);
 cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, int M, int d, float alpha,
                                 int causal, int keep_first, int* row_ptr, int* col_idx, long long capacity,
-                                int* nnz_out, int* row_count, uint32_t* row_bits, cudaStream_t st);
+                                int* nnz_out, int* row_count, uint32_t* row_bits, float* row_max,
+                                cudaStream_t st);
 
 // attn.cu
 struct AttnLaunch {
@@ -52,6 +54,7 @@ struct AttnLaunch {
   const int* row_ptr;   // null in dense mode
   const int* col_idx;   // null in dense mode
   long long col_cap;
+  const float* row_max; // per row max block score (nullable: computed in the kernel)
   uint16_t* out;
   float* lse;
   int BH, N, M, d, causal, dense;

@@ -61,9 +61,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 extern "C" {
 
 int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar,
-                     const float* vsum, const int* row_ptr, const int* col_idx, size_t col_capacity, int B, int H,
-                     int N, int d, int block_size, int causal, psa_bf16_t* out, float* lse, int* status,
-                     void* stream) {
+                     const float* vsum, const int* row_ptr, const int* col_idx, size_t col_capacity,
+                     const float* row_max, int B, int H, int N, int d, int block_size, int causal, psa_bf16_t* out,
+                     float* lse, int* status, void* stream) {
   if (!q || !k || !v || !kbar || !vsum || !row_ptr || !col_idx || !out) return PSA_ERR_ARG;
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return PSA_ERR_ARG;
   if (block_size != psa::kBlock || (d != 64 && d != 128)) return PSA_ERR_UNSUPPORTED;
@@ -73,7 +73,7 @@ int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
   if (causal != 0 && causal != 1) return PSA_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kbar) ||
       !aligned16(vsum) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
-      (status && (reinterpret_cast<uintptr_t>(status) & 3u)))
+      (status && (reinterpret_cast<uintptr_t>(status) & 3u)) || (reinterpret_cast<uintptr_t>(row_max) & 3u))
     return PSA_ERR_ARG;
   const long long bh = static_cast<long long>(B) * H;
   const int M = N / psa::kBlock;
@@ -106,6 +106,7 @@ int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
   a.col_cap = col_capacity > static_cast<size_t>(LLONG_MAX) ? LLONG_MAX : static_cast<long long>(col_capacity);
+  a.row_max = row_max;
   a.out = out;
   a.lse = lse;
   a.BH = static_cast<int>(bh);

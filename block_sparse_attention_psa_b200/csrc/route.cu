@@ -13,7 +13,8 @@
 // selects.  Top-k finds the k-th largest score exactly by a 32-step bitwise
 // search over the order-preserving integer image of the fp32 scores (ties
 // resolved by ascending J), so it needs no sort; both routers write the
-// list in ascending J with warp ballots.
+// list in ascending J with warp ballots, and, when asked, each row's largest
+// candidate score (the attention step's softmax stabiliser).
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
                                                          const float* __restrict__ kbar, int BH, int M, int d,
                                                          float tau, int k0, int causal, int* __restrict__ row_ptr,
                                                          int* __restrict__ col_idx, long long total,
-                                                         int* __restrict__ nnz_out) {
+                                                         int* __restrict__ nnz_out, float* __restrict__ row_max) {
   extern __shared__ float sm[];
   const int bh = blockIdx.y;
   const int I0 = blockIdx.x * R;
@@ -96,6 +97,13 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   // causal: the diagonal takes one slot, the rest come from J < I
   const int n = causal ? I : M;
   const int krest = causal ? kk - 1 : kk;
+  if (row_max) {
+    float m = -INFINITY;
+    for (int J = lane; J < cand; J += 32) m = fmaxf(m, s[J]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) row_max[row] = m;
+  }
 
   uint32_t T = 0;
   if (krest > 0) {
@@ -151,7 +159,8 @@ __global__ void __launch_bounds__(256) route_thresh_kernel(const float* __restri
                                                            const float* __restrict__ kbar, int M, int d,
                                                            float tau, float alpha, int causal, int keep_first,
                                                            int* __restrict__ row_count,
-                                                           uint32_t* __restrict__ row_bits) {
+                                                           uint32_t* __restrict__ row_bits,
+                                                           float* __restrict__ row_max) {
   extern __shared__ float sm[];
   const int bh = blockIdx.y;
   const int I0 = blockIdx.x * R;
@@ -172,6 +181,7 @@ __global__ void __launch_bounds__(256) route_thresh_kernel(const float* __restri
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   const float thr = alpha * m;
+  if (row_max && lane == 0) row_max[row] = m;
   const int nw = (M + 31) / 32;
   uint32_t* bits = row_bits + row * nw;
   int cnt = 0;
@@ -283,7 +293,8 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }  // namespace
 
 cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int M, int d, int k0, int causal,
-                              int* row_ptr, int* col_idx, long long total, int* nnz_out, cudaStream_t st) {
+                              int* row_ptr, int* col_idx, long long total, int* nnz_out, float* row_max,
+                              cudaStream_t st) {
   const int R = rows_per_cta(M, d);
   const size_t smem = static_cast<size_t>(R) * (M + d) * sizeof(float);
   const dim3 grid((M + R - 1) / R, BH);
@@ -293,7 +304,7 @@ cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int 
   case RR:                                                                                             \
     if ((e = set_smem(route_topk_kernel<RR>, smem)) != cudaSuccess) return e;                          \
     route_topk_kernel<RR><<<grid, 256, smem, st>>>(qbar, kbar, BH, M, d, tau, k0, causal, row_ptr,     \
-                                                    col_idx, total, nnz_out);                          \
+                                                    col_idx, total, nnz_out, row_max);                 \
     break;
   switch (R) {
     PSA_TOPK(8)
@@ -309,7 +320,8 @@ cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int 
 
 cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, int M, int d, float alpha,
                                 int causal, int keep_first, int* row_ptr, int* col_idx, long long capacity,
-                                int* nnz_out, int* row_count, uint32_t* row_bits, cudaStream_t st) {
+                                int* nnz_out, int* row_count, uint32_t* row_bits, float* row_max,
+                                cudaStream_t st) {
   const int R = rows_per_cta(M, d);
   const size_t smem = static_cast<size_t>(R) * (M + d) * sizeof(float);
   const dim3 grid((M + R - 1) / R, BH);
@@ -319,7 +331,7 @@ cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, in
   case RR:                                                                                             \
     if ((e = set_smem(route_thresh_kernel<RR>, smem)) != cudaSuccess) return e;                        \
     route_thresh_kernel<RR><<<grid, 256, smem, st>>>(qbar, kbar, M, d, tau, alpha, causal, keep_first, \
-                                                      row_count, row_bits);                            \
+                                                      row_count, row_bits, row_max);                   \
     break;
   switch (R) {
     PSA_THRESH(8)

@@ -49,12 +49,12 @@ def _declare(L: ctypes.CDLL) -> None:
         "psa_workspace_size": (Z, [I, I, I, I]),
         "psa_route_capacity": (Z, [I, I, I, I]),
         "psa_pool": (I, [P, P, P, I, I, I, I, I, P, P, P, P]),
-        "psa_route_topk": (I, [P, P, I, I, I, I, F, I, P, P, Z, P, P]),
-        "psa_route_thresh": (I, [P, P, I, I, I, I, F, I, I, P, P, Z, P, P, Z, P]),
-        "psa_attn": (I, [P, P, P, P, P, P, P, Z, I, I, I, I, I, I, P, P, P, Z, P]),
+        "psa_route_topk": (I, [P, P, I, I, I, I, F, I, P, P, Z, P, P, P]),
+        "psa_route_thresh": (I, [P, P, I, I, I, I, F, I, I, P, P, Z, P, P, P, Z, P]),
+        "psa_attn": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, Z, P]),
         "psa_dense": (I, [P, P, P, I, I, I, I, I, P, P, P, Z, P]),
         "psa_read_status": (I, [P, ctypes.POINTER(I), P]),
-        "psa_attn_noalloc": (I, [P, P, P, P, P, P, P, Z, I, I, I, I, I, I, P, P, P, P]),
+        "psa_attn_noalloc": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -133,43 +133,49 @@ def psa_pool(q, k, v, block_size: int = 64, out=None, stream=None):
     return qbar, kbar, vsum
 
 
+def _route_out(B, H, M, causal, capacity, device):
+    cap = capacity if capacity is not None else psa_route_capacity(B, H, M, causal)
+    return (torch.empty(B * H * M + 1, dtype=torch.int32, device=device),
+            torch.empty(max(cap, 1), dtype=torch.int32, device=device),
+            torch.empty(1, dtype=torch.int32, device=device),
+            torch.empty(B * H * M, dtype=torch.float32, device=device))
+
+
 def psa_route_topk(qbar, kbar, density: float, causal: bool = False, capacity: int | None = None,
                    out=None, stream=None):
-    """Returns (row_ptr, col_idx, nnz) device int32 tensors (nnz has one element)."""
+    """Returns (row_ptr, col_idx, nnz, row_max): device int32 tensors (nnz has
+    one element) and the float32 row maxima of the block scores (``out`` may
+    give row_max as None to skip it)."""
     B, H, M, d = (int(x) for x in qbar.shape)
     if out is None:
-        cap = capacity if capacity is not None else psa_route_capacity(B, H, M, causal)
-        out = (torch.empty(B * H * M + 1, dtype=torch.int32, device=qbar.device),
-               torch.empty(max(cap, 1), dtype=torch.int32, device=qbar.device),
-               torch.empty(1, dtype=torch.int32, device=qbar.device))
-    row_ptr, col_idx, nnz = out
+        out = _route_out(B, H, M, causal, capacity, qbar.device)
+    row_ptr, col_idx, nnz, row_max = out
     _check("psa_route_topk", lib().psa_route_topk(
         _ptr(qbar), _ptr(kbar), B, H, M, d, float(density), int(causal), _ptr(row_ptr), _ptr(col_idx),
-        col_idx.numel(), _ptr(nnz), _stream(stream)))
-    return row_ptr, col_idx, nnz
+        col_idx.numel(), _ptr(nnz), _ptr(row_max), _stream(stream)))
+    return row_ptr, col_idx, nnz, row_max
 
 
 def psa_route_thresh(qbar, kbar, alpha: float, causal: bool = False, keep_first: bool = False,
                      ws=None, capacity: int | None = None, out=None, stream=None):
-    """Returns (row_ptr, col_idx, nnz); nnz > col_idx.numel() means truncated."""
+    """Returns (row_ptr, col_idx, nnz, row_max); nnz > col_idx.numel() means truncated."""
     B, H, M, d = (int(x) for x in qbar.shape)
     if ws is None:
         ws = workspace(B, H, M * 64, d, qbar.device)
     if out is None:
-        cap = capacity if capacity is not None else psa_route_capacity(B, H, M, causal)
-        out = (torch.empty(B * H * M + 1, dtype=torch.int32, device=qbar.device),
-               torch.empty(max(cap, 1), dtype=torch.int32, device=qbar.device),
-               torch.empty(1, dtype=torch.int32, device=qbar.device))
-    row_ptr, col_idx, nnz = out
+        out = _route_out(B, H, M, causal, capacity, qbar.device)
+    row_ptr, col_idx, nnz, row_max = out
     _check("psa_route_thresh", lib().psa_route_thresh(
         _ptr(qbar), _ptr(kbar), B, H, M, d, float(alpha), int(causal), int(keep_first), _ptr(row_ptr),
-        _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(ws), ws.numel(), _stream(stream)))
-    return row_ptr, col_idx, nnz
+        _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(row_max), _ptr(ws), ws.numel(), _stream(stream)))
+    return row_ptr, col_idx, nnz, row_max
 
 
 def psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_size: int = 64,
-             ws=None, out=None, lse=None, want_lse: bool = False, stream=None):
-    """Returns out (bf16 [B,H,N,d]) and, if requested, lse (float32 [B,H,N])."""
+             ws=None, out=None, lse=None, want_lse: bool = False, row_max=None, stream=None):
+    """Returns out (bf16 [B,H,N,d]) and, if requested, lse (float32 [B,H,N]).
+    ``row_max`` (optional) is a router's row maxima, used as the softmax
+    stabiliser instead of computing it in the kernel."""
     B, H, N, d = _shape(q)
     if ws is None:
         ws = workspace(B, H, N, d, q.device)
@@ -179,7 +185,8 @@ def psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_
         lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
     _check("psa_attn", lib().psa_attn(
         _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
-        B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+        _stream(stream)))
     return (out, lse) if lse is not None else out
 
 
@@ -200,7 +207,7 @@ def psa_dense(q, k, v, causal: bool = False, ws=None, out=None, lse=None, want_l
 
 
 def psa_attn_noalloc(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_size: int = 64,
-                     out=None, lse=None, status=None, stream=None):
+                     out=None, lse=None, status=None, row_max=None, stream=None):
     """psa_attn without a workspace, for callers that cannot allocate device
     memory (framework plugins restricted to the framework's own pool, loops
     that forbid allocation after start-up): the library's own 16 MiB scratch
@@ -211,7 +218,8 @@ def psa_attn_noalloc(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False
         out = torch.empty_like(q)
     _check("psa_attn_noalloc", lib().psa_attn_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
-        B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(status), _stream(stream)))
+        _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(status),
+        _stream(stream)))
     return out
 
 
@@ -226,7 +234,7 @@ def psa_forward(q, k, v, mode: str = "topk", density: float = 0.15, alpha: float
                 causal: bool = False, keep_first: bool = False, ws=None, stream=None):
     """The whole path in one call (pool -> route -> attention), as the usage
     line of the PISA summary calls it: f(q, k, v, density=0.15, block_size=64).
-    Returns (out, (row_ptr, col_idx, nnz))."""
+    Returns (out, (row_ptr, col_idx, nnz, row_max))."""
     B, H, N, d = _shape(q)
     if ws is None:
         ws = workspace(B, H, N, d, q.device)
@@ -237,5 +245,5 @@ def psa_forward(q, k, v, mode: str = "topk", density: float = 0.15, alpha: float
         csr = psa_route_thresh(qbar, kbar, alpha, causal, keep_first, ws=ws, stream=stream)
     else:
         raise ValueError("mode must be 'topk' or 'thresh'")
-    out = psa_attn(q, k, v, kbar, vsum, csr[0], csr[1], causal, ws=ws, stream=stream)
+    out = psa_attn(q, k, v, kbar, vsum, csr[0], csr[1], causal, ws=ws, row_max=csr[3], stream=stream)
     return out, csr

@@ -100,15 +100,17 @@ PSA_API int psa_pool(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
  *   blocks: the k highest scores, ties to the smaller J; when causal the
  *   diagonal block takes one of the k slots and the other k-1 are the best
  *   J < I.  Lists ascending.
- * Outputs: row_ptr [B*H*M + 1], col_idx [capacity] (device int32) and
- * *nnz_out (device int32) = total listed.  Errors: PSA_ERR_ARG,
- * PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY (capacity below the exact total,
- * which the host knows for top-k), PSA_ERR_CUDA.
+ * Outputs: row_ptr [B*H*M + 1], col_idx [capacity] (device int32),
+ * *nnz_out (device int32) = total listed, and, when row_max is not NULL,
+ * row_max [B*H*M] (device float32) = max over the candidates of s_IJ, the
+ * softmax stabiliser psa_attn can take instead of computing its own.
+ * Errors: PSA_ERR_ARG, PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY (capacity
+ * below the exact total, which the host knows for top-k), PSA_ERR_CUDA.
  */
 PSA_API int psa_route_topk(const float* qbar, const float* kbar,
                    int B, int H, int M, int d, float density, int causal,
                    int* row_ptr, int* col_idx, size_t capacity, int* nnz_out,
-                   void* stream);
+                   float* row_max, void* stream);
 
 /*
  * a2 + a4. Block scores and sorting-free threshold routing [FlashPrefill
@@ -118,7 +120,8 @@ PSA_API int psa_route_topk(const float* qbar, const float* kbar,
  * Lists ascending.  The total is data dependent: *nnz_out (device) receives
  * the exact total; if it exceeds `capacity`, rows past the capacity are cut
  * (row_ptr stays a valid, truncated CSR) and the caller must retry with a
- * larger col_idx.  psa_route_capacity() never overflows.
+ * larger col_idx.  psa_route_capacity() never overflows.  row_max
+ * (nullable) as for psa_route_topk: the row maxima the threshold is taken of.
  * `workspace` (device, psa_workspace_size(B,H,64*M,d) bytes) holds the row
  * counts and bit masks between the three launches.  Errors: PSA_ERR_ARG,
  * PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY (workspace too small), PSA_ERR_CUDA.
@@ -126,8 +129,8 @@ PSA_API int psa_route_topk(const float* qbar, const float* kbar,
 PSA_API int psa_route_thresh(const float* qbar, const float* kbar,
                      int B, int H, int M, int d, float alpha, int causal,
                      int keep_first, int* row_ptr, int* col_idx, size_t capacity,
-                     int* nnz_out, void* workspace, size_t workspace_bytes,
-                     void* stream);
+                     int* nnz_out, float* row_max, void* workspace,
+                     size_t workspace_bytes, void* stream);
 
 /*
  * a5 - a7. Exact attention on the listed blocks plus the 0th-order term of
@@ -145,6 +148,11 @@ PSA_API int psa_route_thresh(const float* qbar, const float* kbar,
  * col_capacity is the number of int32 entries col_idx points to (a row whose
  * row_ptr range leaves [0, col_capacity] is treated as empty and recorded as
  * PSA_ERR_CSR, so the kernel never reads past the caller's buffer).
+ * row_max (float32 [B*H*M], nullable) is the router's row maximum of s_IJ;
+ * the kernel builds each row's softmax stabiliser from it, and computes the
+ * same quantity itself from q and kbar when it is NULL.  It only shifts the
+ * exponents: any finite values give the same result up to rounding, rows
+ * whose sum would leave the fp32 range are recomputed exactly.
  * Outputs: out bf16 [B,H,N,d]; lse float32 [B,H,N] (may be NULL).
  * A malformed list entry is recorded as PSA_ERR_CSR in the workspace
  * status: an entry out of range (J >= M, or J > I when causal) is skipped,
@@ -155,7 +163,7 @@ PSA_API int psa_route_thresh(const float* qbar, const float* kbar,
 PSA_API int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v,
              const float* kbar, const float* vsum,
              const int* row_ptr, const int* col_idx, size_t col_capacity,
-             int B, int H, int N, int d, int block_size, int causal,
+             const float* row_max, int B, int H, int N, int d, int block_size, int causal,
              psa_bf16_t* out, float* lse,
              void* workspace, size_t workspace_bytes, void* stream);
 
@@ -189,8 +197,8 @@ PSA_API int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t
 PSA_API int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v,
                              const float* kbar, const float* vsum,
                              const int* row_ptr, const int* col_idx, size_t col_capacity,
-                             int B, int H, int N, int d, int block_size, int causal,
-                             psa_bf16_t* out, float* lse, int* status, void* stream);
+                             const float* row_max, int B, int H, int N, int d, int block_size,
+                             int causal, psa_bf16_t* out, float* lse, int* status, void* stream);
 
 /*
  * Synchronises `stream`, then copies the device status word of `workspace`

@@ -29,23 +29,26 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").double().numpy()
 
 
-def run_gpu(q, k, v, mode, param, causal=False, keep_first=False, want_lse=True):
-    """Pool, route and attend on the GPU.  Returns a dict of CPU tensors."""
+def run_gpu(q, k, v, mode, param, causal=False, keep_first=False, want_lse=True, use_row_max=True):
+    """Pool, route and attend on the GPU.  Returns a dict of CPU tensors.
+    ``use_row_max`` hands the router's row maxima to the attention step (as
+    the bench does); otherwise the kernel computes its own stabiliser."""
     dq, dk, dv = (x.cuda() for x in (q, k, v))
     B, H, N, d = q.shape
     ws = psa.workspace(B, H, N, d)
     qbar, kbar, vsum = psa.psa_pool(dq, dk, dv)
     if mode == "topk":
-        row_ptr, col_idx, nnz = psa.psa_route_topk(qbar, kbar, param, causal)
+        row_ptr, col_idx, nnz, row_max = psa.psa_route_topk(qbar, kbar, param, causal)
     else:
-        row_ptr, col_idx, nnz = psa.psa_route_thresh(qbar, kbar, param, causal, keep_first, ws=ws)
-    out, lse = psa.psa_attn(dq, dk, dv, kbar, vsum, row_ptr, col_idx, causal, ws=ws, want_lse=True)
+        row_ptr, col_idx, nnz, row_max = psa.psa_route_thresh(qbar, kbar, param, causal, keep_first, ws=ws)
+    out, lse = psa.psa_attn(dq, dk, dv, kbar, vsum, row_ptr, col_idx, causal, ws=ws, want_lse=True,
+                            row_max=row_max if use_row_max else None)
     status = psa.psa_read_status(ws)
     torch.cuda.synchronize()
     n = int(nnz.item())
     return dict(qbar=qbar.cpu(), kbar=kbar.cpu(), vsum=vsum.cpu(), row_ptr=row_ptr.cpu().long().numpy(),
                 col_idx=col_idx[:n].cpu().long().numpy(), nnz=n, out=out.cpu(), lse=lse.cpu(),
-                status=status)
+                status=status, row_max=row_max.cpu())
 
 
 def check_status(g, want=None):
@@ -88,6 +91,10 @@ def check_routing(g, s, mode, param, causal, keep_first=False):
                 n_cand = I + 1 if causal else M
                 assert got.size == 0 or (got[0] >= 0 and got[-1] < n_cand), f"row {r}: out of range"
                 row = s[b, h, I, :n_cand]
+                if "row_max" in g:
+                    got_max = float(g["row_max"].reshape(-1)[r])
+                    assert abs(got_max - row.max()) <= _band(row.max(), row), \
+                        f"row {r}: row max {got_max}, oracle {row.max()}"
                 if mode == "topk":
                     assert got.size == want.size, f"row {r}: {got.size} listed, want {want.size}"
                     pool_n = I if causal else n_cand

@@ -64,24 +64,31 @@ def test_host_validation_rejects_bad_arguments():
     assert L.psa_pool(ctypes.c_void_p((1 << 20) + 2), FAKE, FAKE, 1, 1, 64, 64, 64, FAKE, FAKE, FAKE, S) \
         == psa.PSA_ERR_ARG
     # top-k: capacity below the exact total, bad density
-    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 2 * 16 * 4 - 1, FAKE, S) \
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 2 * 16 * 4 - 1, FAKE, None, S) \
         == psa.PSA_ERR_CAPACITY
-    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, float("nan"), 0, FAKE, FAKE, 1 << 20, FAKE, S) \
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, float("nan"), 0, FAKE, FAKE, 1 << 20, FAKE, None, S) \
         == psa.PSA_ERR_ARG
-    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 2, FAKE, FAKE, 1 << 20, FAKE, S) == psa.PSA_ERR_ARG
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 2, FAKE, FAKE, 1 << 20, FAKE, None, S) \
+        == psa.PSA_ERR_ARG
     # threshold: workspace too small, bad alpha
-    assert L.psa_route_thresh(FAKE, FAKE, 1, 2, 16, 64, 0.5, 0, 0, FAKE, FAKE, 1 << 20, FAKE, FAKE, 16, S) \
+    assert L.psa_route_thresh(FAKE, FAKE, 1, 2, 16, 64, 0.5, 0, 0, FAKE, FAKE, 1 << 20, FAKE, None, FAKE, 16, S) \
         == psa.PSA_ERR_CAPACITY
-    assert L.psa_route_thresh(FAKE, FAKE, 1, 2, 16, 64, float("inf"), 0, 0, FAKE, FAKE, 1 << 20, FAKE, FAKE,
-                              1 << 30, S) == psa.PSA_ERR_ARG
+    assert L.psa_route_thresh(FAKE, FAKE, 1, 2, 16, 64, float("inf"), 0, 0, FAKE, FAKE, 1 << 20, FAKE, None,
+                              FAKE, 1 << 30, S) == psa.PSA_ERR_ARG
     # attention: workspace too small, misaligned workspace, M too large
     ws = psa.psa_workspace_size(1, 2, 1024, 64)
-    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 1, 2, 1024, 64, 64, 0, FAKE, None, FAKE,
-                      ws - 1, S) == psa.PSA_ERR_CAPACITY
-    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 1, 2, 1024, 64, 64, 0, FAKE, None,
-                      ctypes.c_void_p((1 << 20) + 16), ws, S) == psa.PSA_ERR_ARG
-    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 1, 1, 64 * 16385, 64, 64, 0, FAKE, None,
-                      FAKE, 1 << 40, S) == psa.PSA_ERR_UNSUPPORTED
+    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, None, 1, 2, 1024, 64, 64, 0, FAKE, None,
+                      FAKE, ws - 1, S) == psa.PSA_ERR_CAPACITY
+    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, None, 1, 2, 1024, 64, 64, 0, FAKE,
+                      None, ctypes.c_void_p((1 << 20) + 16), ws, S) == psa.PSA_ERR_ARG
+    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, None, 1, 1, 64 * 16385, 64, 64, 0, FAKE,
+                      None, FAKE, 1 << 40, S) == psa.PSA_ERR_UNSUPPORTED
+    # misaligned row maxima (routers' output, attention's input)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 1 << 20, FAKE, odd, S) \
+        == psa.PSA_ERR_ARG
+    assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, odd, 1, 2, 1024, 64, 64, 0, FAKE,
+                      None, FAKE, ws, S) == psa.PSA_ERR_ARG
     assert L.psa_dense(FAKE, FAKE, FAKE, 1, 2, 1024, 64, 3, FAKE, None, FAKE, ws, S) == psa.PSA_ERR_ARG
     assert L.psa_read_status(None, None, S) == psa.PSA_ERR_ARG
 

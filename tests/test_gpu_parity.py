@@ -213,3 +213,21 @@ def test_full_long_causal_threshold():
 @pytest.mark.parametrize("density", [0.05, 1.0])
 def test_full_sweep(density):
     _full_size("sweep_n64k", density=density, n_units=40)
+
+
+# ------------------------------------------------------------------ stabiliser source
+@pytest.mark.parametrize("causal", [False, True])
+def test_router_row_max_and_kernel_stabiliser_agree(causal):
+    # the stabiliser only shifts exponents: with the router's row maxima and
+    # with the kernel's own, both results match the oracle and each other
+    q, k, v = make_qkv(1, 3, 70 * 64, 128, "clustered", seed=15)
+    g1 = run_gpu(q, k, v, "topk", 0.2, causal, use_row_max=True)
+    g2 = run_gpu(q, k, v, "topk", 0.2, causal, use_row_max=False)
+    qbar, kbar, vsum = check_pool(g1, q, k, v)
+    check_routing(g1, O.block_scores(qbar, kbar), "topk", 0.2, causal)
+    assert np.array_equal(g1["col_idx"], g2["col_idx"])
+    units = sample_units(1, 3, 70, 30, seed=4, g=g1)
+    check_output(g1, q, k, v, kbar, vsum, causal, units)
+    check_output(g2, q, k, v, kbar, vsum, causal, units)
+    err = np.abs(f64(g1["out"]) - f64(g2["out"]))
+    assert err.max() <= 2e-2 and err.mean() <= 1e-3, (err.max(), err.mean())

@@ -29,7 +29,7 @@ def test_no_alloc_matches_workspace_entry_point(causal, d):
     q, k, v = (x.cuda() for x in make_qkv(1, 4, 96 * 64, d, "clustered", seed=21))
     B, H, N, _ = q.shape
     qbar, kbar, vsum = psa.psa_pool(q, k, v)
-    row_ptr, col_idx, _ = psa.psa_route_topk(qbar, kbar, 0.15, causal)
+    row_ptr, col_idx, _, row_max = psa.psa_route_topk(qbar, kbar, 0.15, causal)
     ws = psa.workspace(B, H, N, d)
     ref, ref_lse = psa.psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, causal, ws=ws, want_lse=True)
     assert psa.psa_read_status(ws) == psa.PSA_OK
@@ -42,7 +42,7 @@ def test_no_alloc_matches_workspace_entry_point(causal, d):
             ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
             ctypes.c_void_p(kbar.data_ptr()), ctypes.c_void_p(vsum.data_ptr()),
             ctypes.c_void_p(row_ptr.data_ptr()), ctypes.c_void_p(col_idx.data_ptr()), col_idx.numel(),
-            B, H, N, d, 64, int(causal), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+            None, B, H, N, d, 64, int(causal), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
             ctypes.c_void_p(status.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
         assert rc == psa.PSA_OK, psa.status_text(rc)
         torch.cuda.synchronize()
@@ -58,6 +58,6 @@ def test_no_alloc_rejects_shapes_beyond_its_scratch():
     # B*H*M*d bf16 pairs beyond 16 MiB: rejected on the host, nothing launched
     L = psa.lib()
     fake = ctypes.c_void_p(1 << 20)
-    rc = L.psa_attn_noalloc(fake, fake, fake, fake, fake, fake, fake, 1 << 20, 1, 64, 65536, 128, 64, 0,
+    rc = L.psa_attn_noalloc(fake, fake, fake, fake, fake, fake, fake, 1 << 20, None, 1, 64, 65536, 128, 64, 0,
                             fake, None, None, None)
     assert rc == psa.PSA_ERR_CAPACITY
