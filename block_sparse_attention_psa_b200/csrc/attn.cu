@@ -506,8 +506,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (abort raised) they return at once and the group runs on with garbage
     // data until the next unit boundary, where all 256 threads take the same
     // stop decision.  This keeps every named barrier matched.
-    // turn-taking for the exponentials: warpgroup 0 owns tile 0, so it starts
-    if (w == 1) named_barrier_arrive(2, 256);
     float c2 = 0.f;  // stabiliser of the current unit (log2 units)
     int sc = 0;   // running tile index (both warpgroups count every tile)
     int my = 0;   // tiles of this warpgroup so far (S buffer phase)
@@ -641,10 +639,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // warp-uniform except the pooled-key validity, which is a select
         const int mode = pseudo ? 1 : (!valid ? 3 : (diag ? 2 : 0));
         const int kj = trow & 63;
-        // The two warpgroups share the special-function units: they take
-        // turns (tile parity order) for the exponentials, so one warpgroup's
-        // exponentials overlap the other's loads, stores and waits.
-        named_barrier_sync(2 + w, 256);
         uint32_t pk[32];
         if (mode == 0) {
           exp_half<0, 0>(sv, bias, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
@@ -659,7 +653,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) pk[i] = 0u;
         }
-        named_barrier_arrive(2 + (w ^ 1), 256);
         // P^T row of this thread: 64 bf16 as eight 16-byte chunks (128-byte
         // swizzle: chunk c lands at c ^ (row % 8)), once this warpgroup's
         // previous GEMM2 has finished reading the buffer
@@ -712,8 +705,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // the last tile's owner handed the turn to the other warpgroup: take it
-    if ((sc & 1) == w) named_barrier_sync(2 + w, 256);
     if (gtid == 0) bulk_wait0();
   }
 

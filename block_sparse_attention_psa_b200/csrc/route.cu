@@ -40,41 +40,85 @@ __host__ __device__ inline long long causal_prefix(long long I, long long k0) {
 }
 
 // Scores of rows [I0, I0 + rows) of head bh into ss[r * M + J], J < jmax.
-template <int R>
+// Thread t owns key J0 + t of each 256-key chunk and accumulates its R dot
+// products over the features in order.  The kbar rows reach it through
+// shared memory, 16 features of 256 keys at a time: loaded with coalesced
+// 16-byte loads (read straight from global memory, every lane of a warp
+// would touch a different cache line) into rows padded to 20 floats, so the
+// per-thread 16-byte reads are free of bank conflicts.  The next slice is
+// fetched into registers while the current one is consumed.
+constexpr int kSliceF = 16;            // features per slice
+constexpr int kSliceStride = 20;       // padded row, floats
+constexpr int kChunkJ = 256;           // keys per chunk (one per thread)
+
+template <int R, int D>
 __device__ void score_rows(const float* __restrict__ qbar, const float* __restrict__ kbar, int bh, int M,
-                           int d, int I0, int rows, int jmax, float tau, float* sq, float* ss) {
-  for (int e = threadIdx.x; e < R * d; e += blockDim.x)
-    sq[e] = e < rows * d ? qbar[(static_cast<size_t>(bh) * M + I0) * d + e] : 0.f;
-  __syncthreads();
-  const float* kb = kbar + static_cast<size_t>(bh) * M * d;
+                           int I0, int rows, int jmax, float tau, float* sq, float* sk, float* ss) {
+  static_assert(D % kSliceF == 0, "slices");
+  constexpr int kSlices = D / kSliceF;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < R * D; e += blockDim.x)
+    sq[e] = e < rows * D ? qbar[(static_cast<size_t>(bh) * M + I0) * D + e] : 0.f;
+  const float* kb = kbar + static_cast<size_t>(bh) * M * D;
   const float4* sq4 = reinterpret_cast<const float4*>(sq);
-  const int d4 = d / 4;
-  for (int J = threadIdx.x; J < jmax; J += blockDim.x) {
+  for (int J0 = 0; J0 < jmax; J0 += kChunkJ) {
+    // slice loader: float4 e = i * 256 + tid covers key row e / 4, features 4 (e % 4) ..
+    float4 pre[4];
+    auto fetch = [&](int s) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = i * 256 + tid, row = e >> 2, c4 = e & 3;
+        pre[i] = J0 + row < jmax
+                     ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(J0 + row) * D + s * kSliceF) + c4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    auto stash = [&](float* buf) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = i * 256 + tid, row = e >> 2, c4 = e & 3;
+        *reinterpret_cast<float4*>(buf + row * kSliceStride + 4 * c4) = pre[i];
+      }
+    };
     float acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
-    const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<size_t>(J) * d);
-    for (int c = 0; c < d4; ++c) {
-      const float4 kv = __ldg(kr + c);
+    fetch(0);
+    __syncthreads();  // previous chunk's readers are done with both buffers
+    stash(sk);
+#pragma unroll 1
+    for (int s = 0; s < kSlices; ++s) {
+      float* cur = sk + (s & 1) * kChunkJ * kSliceStride;
+      if (s + 1 < kSlices) fetch(s + 1);
+      __syncthreads();
+      const float4* kr = reinterpret_cast<const float4*>(cur + tid * kSliceStride);
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float4 qv = sq4[r * d4 + c];
-        acc[r] = fmaf(qv.x, kv.x, acc[r]);
-        acc[r] = fmaf(qv.y, kv.y, acc[r]);
-        acc[r] = fmaf(qv.z, kv.z, acc[r]);
-        acc[r] = fmaf(qv.w, kv.w, acc[r]);
+      for (int c = 0; c < kSliceF / 4; ++c) {
+        const float4 kv = kr[c];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const float4 qv = sq4[r * (D / 4) + s * (kSliceF / 4) + c];
+          acc[r] = fmaf(qv.x, kv.x, acc[r]);
+          acc[r] = fmaf(qv.y, kv.y, acc[r]);
+          acc[r] = fmaf(qv.z, kv.z, acc[r]);
+          acc[r] = fmaf(qv.w, kv.w, acc[r]);
+        }
       }
+      if (s + 1 < kSlices) stash(sk + ((s + 1) & 1) * kChunkJ * kSliceStride);
     }
+    const int J = J0 + tid;
+    if (J < jmax) {
 #pragma unroll
-    for (int r = 0; r < R; ++r)
-      if (r < rows) ss[r * M + J] = acc[r] * tau + 0.0f;  // +0 folds -0 into +0
+      for (int r = 0; r < R; ++r)
+        if (r < rows) ss[r * M + J] = acc[r] * tau + 0.0f;  // +0 folds -0 into +0
+    }
   }
   __syncthreads();
 }
 
-template <int R>
+template <int R, int D>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ qbar,
-                                                         const float* __restrict__ kbar, int BH, int M, int d,
+                                                         const float* __restrict__ kbar, int BH, int M,
                                                          float tau, int k0, int causal, int* __restrict__ row_ptr,
                                                          int* __restrict__ col_idx, long long total,
                                                          int* __restrict__ nnz_out, float* __restrict__ row_max) {
@@ -84,8 +128,9 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   const int rows = min(R, M - I0);
   const int jmax = causal ? min(M, I0 + rows) : M;
   float* sq = sm;
-  float* ss = sm + R * d;
-  score_rows<R>(qbar, kbar, bh, M, d, I0, rows, jmax, tau, sq, ss);
+  float* sk = sq + R * D;
+  float* ss = sk + 2 * kChunkJ * kSliceStride;
+  score_rows<R, D>(qbar, kbar, bh, M, I0, rows, jmax, tau, sq, sk, ss);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (warp >= rows) return;
@@ -154,9 +199,9 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   }
 }
 
-template <int R>
+template <int R, int D>
 __global__ void __launch_bounds__(256) route_thresh_kernel(const float* __restrict__ qbar,
-                                                           const float* __restrict__ kbar, int M, int d,
+                                                           const float* __restrict__ kbar, int M,
                                                            float tau, float alpha, int causal, int keep_first,
                                                            int* __restrict__ row_count,
                                                            uint32_t* __restrict__ row_bits,
@@ -167,8 +212,9 @@ __global__ void __launch_bounds__(256) route_thresh_kernel(const float* __restri
   const int rows = min(R, M - I0);
   const int jmax = causal ? min(M, I0 + rows) : M;
   float* sq = sm;
-  float* ss = sm + R * d;
-  score_rows<R>(qbar, kbar, bh, M, d, I0, rows, jmax, tau, sq, ss);
+  float* sk = sq + R * D;
+  float* ss = sk + 2 * kChunkJ * kSliceStride;
+  score_rows<R, D>(qbar, kbar, bh, M, I0, rows, jmax, tau, sq, sk, ss);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (warp >= rows) return;
@@ -278,10 +324,14 @@ __global__ void __launch_bounds__(256) compact_rows_kernel(const uint32_t* __res
   }
 }
 
+// shared memory of a router CTA: R query rows, the two kbar slices, R score rows
+size_t route_smem(int R, int M, int d) {
+  return (static_cast<size_t>(R) * (M + d) + 2 * kChunkJ * kSliceStride) * sizeof(float);
+}
+
 int rows_per_cta(int M, int d) {
-  // scores of R rows plus R query rows must fit in ~200 KB of shared memory
   for (int R = 8; R > 1; R >>= 1)
-    if (static_cast<size_t>(R) * (M + d) * sizeof(float) <= 200 * 1024) return R;
+    if (route_smem(R, M, d) <= 200 * 1024) return R;
   return 1;
 }
 
@@ -296,16 +346,23 @@ cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int 
                               int* row_ptr, int* col_idx, long long total, int* nnz_out, float* row_max,
                               cudaStream_t st) {
   const int R = rows_per_cta(M, d);
-  const size_t smem = static_cast<size_t>(R) * (M + d) * sizeof(float);
+  const size_t smem = route_smem(R, M, d);
   const dim3 grid((M + R - 1) / R, BH);
   const float tau = 1.0f / sqrtf(static_cast<float>(d));
   cudaError_t e;
 #define PSA_TOPK(RR)                                                                                   \
   case RR:                                                                                             \
-    if ((e = set_smem(route_topk_kernel<RR>, smem)) != cudaSuccess) return e;                          \
-    route_topk_kernel<RR><<<grid, 256, smem, st>>>(qbar, kbar, BH, M, d, tau, k0, causal, row_ptr,     \
-                                                    col_idx, total, nnz_out, row_max);                 \
+    if (d == 128) {                                                                                    \
+      if ((e = set_smem(route_topk_kernel<RR, 128>, smem)) != cudaSuccess) return e;                   \
+      route_topk_kernel<RR, 128><<<grid, 256, smem, st>>>(qbar, kbar, BH, M, tau, k0, causal, row_ptr, \
+                                                           col_idx, total, nnz_out, row_max);          \
+    } else {                                                                                           \
+      if ((e = set_smem(route_topk_kernel<RR, 64>, smem)) != cudaSuccess) return e;                    \
+      route_topk_kernel<RR, 64><<<grid, 256, smem, st>>>(qbar, kbar, BH, M, tau, k0, causal, row_ptr,  \
+                                                          col_idx, total, nnz_out, row_max);           \
+    }                                                                                                  \
     break;
+  if (d != 64 && d != 128) return cudaErrorInvalidValue;
   switch (R) {
     PSA_TOPK(8)
     PSA_TOPK(4)
@@ -323,16 +380,23 @@ cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, in
                                 int* nnz_out, int* row_count, uint32_t* row_bits, float* row_max,
                                 cudaStream_t st) {
   const int R = rows_per_cta(M, d);
-  const size_t smem = static_cast<size_t>(R) * (M + d) * sizeof(float);
+  const size_t smem = route_smem(R, M, d);
   const dim3 grid((M + R - 1) / R, BH);
   const float tau = 1.0f / sqrtf(static_cast<float>(d));
   cudaError_t e;
 #define PSA_THRESH(RR)                                                                                 \
   case RR:                                                                                             \
-    if ((e = set_smem(route_thresh_kernel<RR>, smem)) != cudaSuccess) return e;                        \
-    route_thresh_kernel<RR><<<grid, 256, smem, st>>>(qbar, kbar, M, d, tau, alpha, causal, keep_first, \
-                                                      row_count, row_bits, row_max);                   \
+    if (d == 128) {                                                                                    \
+      if ((e = set_smem(route_thresh_kernel<RR, 128>, smem)) != cudaSuccess) return e;                 \
+      route_thresh_kernel<RR, 128><<<grid, 256, smem, st>>>(qbar, kbar, M, tau, alpha, causal,         \
+                                                             keep_first, row_count, row_bits, row_max); \
+    } else {                                                                                           \
+      if ((e = set_smem(route_thresh_kernel<RR, 64>, smem)) != cudaSuccess) return e;                  \
+      route_thresh_kernel<RR, 64><<<grid, 256, smem, st>>>(qbar, kbar, M, tau, alpha, causal,          \
+                                                            keep_first, row_count, row_bits, row_max);  \
+    }                                                                                                  \
     break;
+  if (d != 64 && d != 128) return cudaErrorInvalidValue;
   switch (R) {
     PSA_THRESH(8)
     PSA_THRESH(4)
