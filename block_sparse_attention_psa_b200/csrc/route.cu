@@ -157,7 +157,12 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
       int cnt = 0;
       for (int J = lane; J < n; J += 32) cnt += order_key(s[J]) >= t;
       cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= krest) T = t;
+      if (cnt >= krest) {
+        T = t;
+        // exactly krest keys are >= T: they are the selection (every key equal
+        // to T is in it, so the tie rule below takes them all)
+        if (cnt == krest) break;
+      }
     }
   }
   int gt = 0;

@@ -11,7 +11,7 @@ import torch
 import oracle.psa_oracle as O
 from block_sparse_attention_psa_b200 import psa
 from block_sparse_attention_psa_b200.inputs import WORKLOADS, make_qkv, workload_inputs
-from tests.parity import (check_output, check_pool, check_routing, f64, run_gpu, sample_units)
+from tests.parity import (check_output, check_pool, check_routing, check_status, f64, run_gpu, sample_units)
 
 pytestmark = pytest.mark.gpu
 
@@ -231,3 +231,25 @@ def test_router_row_max_and_kernel_stabiliser_agree(causal):
     check_output(g2, q, k, v, kbar, vsum, causal, units)
     err = np.abs(f64(g1["out"]) - f64(g2["out"]))
     assert err.max() <= 2e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_topk_ties_go_to_smaller_blocks(causal):
+    # every key block has the same pooled key, so every score of a row ties:
+    # the k slots go to the smallest J (the causal diagonal keeps its own slot)
+    B, H, M, d = 1, 2, 40, 64
+    q, _, v = make_qkv(B, H, M * 64, d, "iid", seed=16)
+    k = torch.ones(B, H, M * 64, d, dtype=torch.bfloat16) * 0.5
+    g = run_gpu(q, k, v, "topk", 0.2, causal)
+    check_status(g)
+    kk = int(np.ceil(np.float32(0.2) * np.float32(M)))
+    rp, ci = g["row_ptr"], g["col_idx"]
+    for r in range(B * H * M):
+        I = r % M
+        got = list(ci[rp[r]:rp[r + 1]])
+        if causal:
+            n = min(kk, I + 1)
+            want = sorted(set(range(n - 1)) | {I})
+        else:
+            want = list(range(kk))
+        assert got == want, (r, got, want)
