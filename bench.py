@@ -94,7 +94,7 @@ class ClockSampler:
 
     def start(self):
         cmd = ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
-               "-lms", "200"]
+               "-lms", "50"]
         if self.target:
             cmd += ["--id=" + str(self.target)]
         try:
@@ -135,9 +135,10 @@ class ClockSampler:
 class Step:
     """Device buffers and one step of the path for one workload."""
 
-    def __init__(self, name, density, seed, device):
+    def __init__(self, name, density, seed, device, dense=False):
         w = dict(WORKLOADS[name])
         self.name = name
+        self.dense = dense  # psa_dense (every candidate exact) instead of pool -> route -> attn
         self.w = w
         self.B, self.H, self.N, self.d = w["B"], w["H"], w["N"], w["d"]
         self.M = self.N // 64
@@ -164,11 +165,21 @@ class Step:
         self.out_host = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
         self.stream = torch.cuda.current_stream()
         # kernels of ours launched by one step
-        self.launches = 1 + (1 if self.mode == "topk" else 3) + 3
+        self.launches = 3 if dense else 1 + (1 if self.mode == "topk" else 3) + 3
 
     def run(self, ev=None):
         """pool -> route -> attention; ``ev`` = 4 events to split the kernels."""
         s = self.stream
+        if self.dense:
+            # the dense baseline: one call (it pools the keys for its stabiliser itself)
+            if ev:
+                ev[0].record(s)
+                ev[1].record(s)
+                ev[2].record(s)
+            psa.psa_dense(self.q, self.k, self.v, self.causal, ws=self.ws, out=self.out, stream=s)
+            if ev:
+                ev[3].record(s)
+            return
         if ev:
             ev[0].record(s)
         psa.psa_pool(self.q, self.k, self.v, out=self.stats, stream=s)
@@ -252,7 +263,7 @@ def gpu_arm(args):
     if args.gpus != world and world > 1:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
     device = torch.device("cuda", local)
-    st = Step(args.workload, args.density, seed=rank, device=device)
+    st = Step(args.workload, args.density, seed=rank, device=device, dense=args.dense)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     for _ in range(args.warmup):
         st.run()
@@ -260,12 +271,19 @@ def gpu_arm(args):
     torch.cuda.synchronize()
 
     # routing of this batch, for the executed-FLOP count and density
-    rp = st.csr[0].cpu().numpy()
-    nnz = int(st.csr[2].item())
-    ci = st.csr[1][:nnz].cpu().numpy()
-    ex_flops = executed_flops(rp, ci, st.B, st.H, st.M, st.d, st.causal)
-    de_flops = dense_flops(st.B, st.H, st.N, st.d, st.causal)
     n_cand = st.B * st.H * (st.M * (st.M + 1) // 2 if st.causal else st.M * st.M)
+    if st.dense:
+        rows = st.B * st.H * st.M
+        nsel = np.tile(np.arange(1, st.M + 1) if st.causal else np.full(st.M, st.M), st.B * st.H)
+        rp = np.concatenate([[0], np.cumsum(nsel)])
+        nnz = n_cand
+        ex_flops = executed_flops(rp, None, st.B, st.H, st.M, st.d, st.causal)
+        assert rp[-1] == nnz and len(rp) == rows + 1
+    else:
+        rp = st.csr[0].cpu().numpy()
+        nnz = int(st.csr[2].item())
+        ex_flops = executed_flops(rp, None, st.B, st.H, st.M, st.d, st.causal)
+    de_flops = dense_flops(st.B, st.H, st.N, st.d, st.causal)
     status = psa.psa_read_status(st.ws)
 
     clocks = ClockSampler(local)
@@ -319,17 +337,20 @@ def gpu_arm(args):
         "dtype": "bf16",
         "data": "synthetic (seeded generator, seed = rank)",
         "config": {"workload": st.name, "B": st.B, "H": st.H, "N": st.N, "d": st.d, "block": 64,
-                   "causal": st.causal, "routing": f"{st.mode} {st.param}", "keep_first": st.keep_first,
+                   "causal": st.causal, "routing": "dense (psa_dense)" if st.dense else f"{st.mode} {st.param}",
+                   "keep_first": st.keep_first,
                    "parallelism": f"replicas x{world} (independent problems)" if world > 1 else "1 GPU",
                    "l2": "flushed between steps (512 MB write outside the timed events)"},
-        "roofline": {"bound": "tensor", "kernel": "attn_kernel (psa_attn call)",
+        "roofline": {"bound": "tensor",
+                     "kernel": "attn_kernel (psa_dense call)" if st.dense else "attn_kernel (psa_attn call)",
                      "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": round(achieved / tc_peak, 4), "traffic": recorded_traffic(st.name),
                      "peak_source": peaks["source"] + " bf16 burst"},
-        "kernels": {"pool_ms": round(pool_avg, 4), "route_ms": round(route_avg, 4), "attn_ms": round(attn_avg, 4),
-                    "pool_gbs": round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3) / 1e9, 1),
-                    "pool_hbm_frac": round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3) / 1e9
-                                           / peaks["hbm_gbs"], 4),
+        "kernels": {"pool_ms": None if st.dense else round(pool_avg, 4),
+                    "route_ms": None if st.dense else round(route_avg, 4), "attn_ms": round(attn_avg, 4),
+                    "pool_gbs": None if st.dense else round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3) / 1e9, 1),
+                    "pool_hbm_frac": None if st.dense else round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3)
+                                                                 / 1e9 / peaks["hbm_gbs"], 4),
                     "attn_executed_tflops": round(achieved, 2),
                     "attn_effective_tflops": round(de_flops / (attn_avg * 1e-3) / 1e12, 2)},
         "flops": {"dense_equivalent": de_flops, "executed": ex_flops},
@@ -342,6 +363,8 @@ def gpu_arm(args):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the oracle's sparse step at this workload's routing (also for --dense: the
+        # oracle has no separate dense path; density 1.0 of the sweep is its dense case)
         line["cpu_baseline"] = cpu_baseline(st.name, st.param, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -495,6 +518,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dense", action="store_true", help="time psa_dense (density 1, every block exact) instead")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
