@@ -71,6 +71,23 @@ def executed_flops(row_ptr, col_idx, B, H, M, d, causal):
     return 4.0 * d * exact_pairs + 4.0 * d * b * unlisted.sum()
 
 
+def issued_flops(row_ptr, B, H, M, d, causal, dense=False):
+    """FLOPs the attention kernel's MMAs issue (host, from the block lists):
+    per tile S^T = K Q^T (128 x 64 x d) and O^T += V^T P^T (128 x 64 x 128,
+    M = 128 rows even when d = 64).  A unit takes ceil(listed / 2) exact tiles
+    and, when some candidate is unlisted, ceil(pooled candidates / 128) pooled
+    tiles (at least one tile in all)."""
+    rp = row_ptr.astype(np.int64)
+    nsel = np.diff(rp)
+    I = np.arange(B * H * M) % M
+    cand = I + 1 if causal else np.full_like(I, M)
+    pcand = I if causal else np.full_like(I, M)
+    n_a2 = np.where((~np.bool_(dense)) & (pcand > 0) & (nsel < cand), (pcand + 127) // 128, 0)
+    n_e = (nsel + 1) // 2
+    tiles = np.maximum(n_a2 + n_e, 1)
+    return float(tiles.sum()) * (2.0 * 128 * 64 * d + 2.0 * 128 * 64 * 128)
+
+
 def pool_bytes(B, H, N, d):
     M = N // 64
     return 3 * B * H * N * d * 2 + 3 * B * H * M * d * 4
@@ -278,11 +295,13 @@ def gpu_arm(args):
         rp = np.concatenate([[0], np.cumsum(nsel)])
         nnz = n_cand
         ex_flops = executed_flops(rp, None, st.B, st.H, st.M, st.d, st.causal)
+        is_flops = issued_flops(rp, st.B, st.H, st.M, st.d, st.causal, dense=True)
         assert rp[-1] == nnz and len(rp) == rows + 1
     else:
         rp = st.csr[0].cpu().numpy()
         nnz = int(st.csr[2].item())
         ex_flops = executed_flops(rp, None, st.B, st.H, st.M, st.d, st.causal)
+        is_flops = issued_flops(rp, st.B, st.H, st.M, st.d, st.causal)
     de_flops = dense_flops(st.B, st.H, st.N, st.d, st.causal)
     status = psa.psa_read_status(st.ws)
 
@@ -353,7 +372,8 @@ def gpu_arm(args):
                                                                  / 1e9 / peaks["hbm_gbs"], 4),
                     "attn_executed_tflops": round(achieved, 2),
                     "attn_effective_tflops": round(de_flops / (attn_avg * 1e-3) / 1e12, 2)},
-        "flops": {"dense_equivalent": de_flops, "executed": ex_flops},
+        "flops": {"dense_equivalent": de_flops, "executed": ex_flops, "mma_issued": is_flops,
+                  "mma_issued_tflops": round(is_flops / (attn_avg * 1e-3) / 1e12, 2)},
         "density": {"realised": round(nnz / n_cand, 5), "listed_blocks": nnz},
         "device_status": status,
         "e2e": {"value": round(weak_scaling_value(de_flops, world, e2e_ms), 3), "unit": "TFLOP/s",

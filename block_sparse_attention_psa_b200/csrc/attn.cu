@@ -197,17 +197,7 @@ __device__ __forceinline__ void reg_alloc() {
 // block; 1: pooled key of an unlisted block (weight 64 e^{a-c}, masked by
 // `keep`); 2: diagonal block under the causal mask (key kj visible to query
 // q iff kj <= q).
-// Query pairs (bit i = queries 2i, 2i+1 of a half) whose exponentials are
-// computed on the FMA pipe instead of the special-function unit.
-#ifndef PSA_POLY_PAIRS
-#define PSA_POLY_PAIRS 0x0u
-#endif
-// Packed fp32 pair instructions for the scale/bias and the denominators.
-#ifndef PSA_F32X2
-#define PSA_F32X2 1
-#endif
-constexpr uint32_t kPolyPairs = PSA_POLY_PAIRS;
-
+// The scale/bias and the denominator sums use packed fp32 pair instructions.
 template <int kMode, int kHalf>
 __device__ __forceinline__ void exp_half(const float (&sv)[64], float bias, float (&lsum)[64], float sl, int kj,
                                          bool keep, uint32_t (&pk)[16]) {
@@ -215,40 +205,18 @@ __device__ __forceinline__ void exp_half(const float (&sv)[64], float bias, floa
   for (int i = 0; i < 16; ++i) {
     const int q0 = 32 * kHalf + 2 * i, q1 = q0 + 1;
     float x0, x1;
-#if PSA_F32X2
     ffma2(x0, x1, sv[q0], sv[q1], sl, sl, bias, bias);
-#else
-    x0 = fmaf(sv[q0], sl, bias);
-    x1 = fmaf(sv[q1], sl, bias);
-#endif
-    float e0, e1;
-    if ((kPolyPairs >> i) & 1u) {
-      e0 = exp2_poly(x0);
-      e1 = exp2_poly(x1);
-    } else {
-      e0 = ex2_approx(x0);
-      e1 = ex2_approx(x1);
-    }
+    float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
     if (kMode == 1) {
       e0 = keep ? e0 : 0.f;
       e1 = keep ? e1 : 0.f;
-#if PSA_F32X2
       ffma2(lsum[q0], lsum[q1], e0, e1, 64.f, 64.f, lsum[q0], lsum[q1]);
-#else
-      lsum[q0] = fmaf(e0, 64.f, lsum[q0]);
-      lsum[q1] = fmaf(e1, 64.f, lsum[q1]);
-#endif
     } else {
       if (kMode == 2) {
         e0 = kj <= q0 ? e0 : 0.f;
         e1 = kj <= q1 ? e1 : 0.f;
       }
-#if PSA_F32X2
       fadd2(lsum[q0], lsum[q1], lsum[q0], lsum[q1], e0, e1);
-#else
-      lsum[q0] += e0;
-      lsum[q1] += e1;
-#endif
     }
     pk[i] = pack_bf16x2(e0, e1);
   }

@@ -233,23 +233,6 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// 2^x on the FMA pipe (offloads the special-function unit).  x = n + f with
-// n = round(x) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial fitted for
-// minimum relative error (7.5e-5, from gen_exp2_poly.py), 2^n by adding n to
-// the exponent field.  x is clamped to [-126, 126] so the exponent add can
-// neither wrap nor leave the normal range: results below 2^-126 are
-// negligible here, and a clamped large x still yields a sum above the range
-// the attention kernel accepts (its row is recomputed exactly).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fminf(fmaxf(x, -126.0f), 126.0f);
-  const float t = x + 12582912.0f;  // 1.5 * 2^23: round(x) lands in the low mantissa bits
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(5.517166681e-02f, f, 2.426111351e-01f);
-  p = fmaf(p, f, 6.932609870e-01f);
-  p = fmaf(p, f, 9.999280728e-01f);
-  // (bits(t) - bits(1.5 * 2^23)) << 23 == bits(t) << 23 modulo 2^32
-  return __int_as_float(__float_as_int(t) * 8388608 + __float_as_int(p));
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

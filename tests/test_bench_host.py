@@ -1,0 +1,59 @@
+"""Host-side FLOP accounting of bench.py against brute-force counts (CPU)."""
+
+import numpy as np
+import pytest
+
+import bench
+
+
+def _brute_executed(lists, M, d, causal, b=64):
+    """Count multiply-adds pair by pair: every visible (query, key) token pair of a
+    listed block, and every (query, unlisted candidate block) pseudo-key, at 4 d FLOPs."""
+    pairs = 0
+    r = 0
+    for I in range(M):
+        listed = set(lists[r])
+        cand = range(I + 1) if causal else range(M)
+        for J in cand:
+            if J in listed:
+                for i in range(b):
+                    for j in range(b):
+                        if not causal or J < I or j <= i:
+                            pairs += 1
+            elif not (causal and J == I):
+                pairs += b  # one pseudo-key per query of the block
+        r += 1
+    return 4.0 * d * pairs
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_executed_flops_matches_pair_count(causal):
+    rng = np.random.default_rng(3)
+    M, d = 6, 8
+    lists = []
+    for I in range(M):
+        n = I + 1 if causal else M
+        keep = rng.random(n) < 0.5
+        if causal:
+            keep[I] = True  # the routers always list the causal diagonal
+        lists.append(np.nonzero(keep)[0])
+    rp = np.concatenate([[0], np.cumsum([len(x) for x in lists])])
+    got = bench.executed_flops(rp, None, 1, 1, M, d, causal)
+    assert got == _brute_executed(lists, M, d, causal)
+
+
+def test_issued_flops_counts_tiles():
+    # M = 4 non-causal, list sizes 0, 1, 4, 3: tiles 1 (pooled only), 1 + 1,
+    # 2 (everything listed: no pooled tile), 1 + 2 -> 8 tiles
+    rp = np.array([0, 0, 1, 5, 8])
+    per_tile = 2.0 * 128 * 64 * 128 + 2.0 * 128 * 64 * 128
+    assert bench.issued_flops(rp, 1, 1, 4, 128, False) == 8 * per_tile
+    # dense: every candidate listed, no pooled tiles; causal row I lists I + 1 blocks
+    rp_dense = np.concatenate([[0], np.cumsum(np.arange(1, 5))])
+    assert bench.issued_flops(rp_dense, 1, 1, 4, 64, True, dense=True) == \
+        (1 + 1 + 2 + 2) * (2.0 * 128 * 64 * 64 + 2.0 * 128 * 64 * 128)
+
+
+def test_dense_flops_formula():
+    assert bench.dense_flops(2, 3, 128, 64, False) == 4.0 * 2 * 3 * 128 * 128 * 64
+    assert bench.dense_flops(2, 3, 128, 64, True) == 2.0 * 2 * 3 * 128 * 128 * 64
