@@ -479,101 +479,110 @@ __global__ void __launch_bounds__(kThreads, 1)
     int my = 0;   // tiles of this warpgroup so far (S buffer phase)
     int mp = 0;   // P^T tiles written by this warpgroup so far (P buffer phase)
     int ul = 0;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++ul) {
-      named_barrier_sync(1, 256);
-      if (gtid == 0) *stop_s = *abort_flag;
-      named_barrier_sync(1, 256);
-      if (*stop_s) break;
-      const Unit x = make_unit(u, p);
-      if (!p.dense) {
-        // mark the listed blocks (A2 skips them), cache the list, validate it
-        const int nw = (x.cand + 31) / 32;
-        for (int i = gtid; i < nw; i += 256) bitmap[i] = 0u;
+    Unit x;
+    float bias = 0.f;
+    // Start of a unit: the group-consistent stop decision, the unit's block
+    // list (bitmap of listed blocks for the pooled tiles, cached list) and
+    // its stabiliser.  Returns false when the kernel is stopping.
+    auto prologue = [&](int u) -> bool {
         named_barrier_sync(1, 256);
-        bool bad = x.bad;
-        for (int i = gtid; i < x.nsel; i += 256) {
-          const int J = __ldg(p.col_idx + x.rp + i);
-          if (i < kColCache) cols[i] = J;
-          if (J < 0 || J >= x.cand) {
-            bad = true;
-          } else {
-            const uint32_t bit = 1u << (J & 31);
-            if (atomicOr(&bitmap[J >> 5], bit) & bit) bad = true;
-          }
-        }
-        if (bad) record_status(p.status, kStatusCsr);
+        if (gtid == 0) *stop_s = *abort_flag;
         named_barrier_sync(1, 256);
-      }
-#pragma unroll
-      for (int q = 0; q < 64; ++q) lsum[q] = 0.f;
-      // Stabiliser of the whole query block (log2 units): c2 = max over the
-      // candidate blocks of qbar_I . kbar_J / sqrt(d) * log2(e) + log2(64),
-      // with qbar_I the mean of the block's queries.  Any constant within a
-      // few tens of the rows' largest logits keeps every term in range; rows
-      // whose sum still leaves [2^-60, 2^60] are recomputed by the fixup.
-      if (p.row_max) {
-        // the router's largest block score of this row, qbar_I . kbar_J / sqrt(d)
-        c2 = __ldg(p.row_max + x.row) * 1.4426950408889634f + 6.0f;
-      } else {
-        constexpr int kCh = D / 8;             // 16-byte chunks of a row
-        constexpr int kGr = 256 / kCh;         // row groups
-        const int ch = gtid % kCh, gr = gtid / kCh;
-        const uint4* qrow = reinterpret_cast<const uint4*>(p.q) + (static_cast<size_t>(x.row) * 64) * kCh + ch;
-        float part[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) part[i] = 0.f;
-#pragma unroll
-        for (int r = gr; r < 64; r += kGr) {
-          const uint4 w4 = __ldg(qrow + static_cast<size_t>(r) * kCh);
-          const uint32_t u[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            part[2 * i] += __uint_as_float(u[i] << 16);
-            part[2 * i + 1] += __uint_as_float(u[i] & 0xffff0000u);
-          }
-        }
-#pragma unroll
-        for (int o = kCh; o < 32; o <<= 1)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
-        if (lane < kCh) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) red[gwarp * 64 * 2 + ch * 8 + i] = part[i];  // [8 warps][<=128]
-        }
-        named_barrier_sync(1, 256);
-        if (gtid < D) {
-          float sum = 0.f;
-#pragma unroll
-          for (int wv = 0; wv < 8; ++wv) sum += red[wv * 128 + gtid];
-          qbs[gtid] = sum * (1.0f / 64.0f);
-        }
-        named_barrier_sync(1, 256);
-        float mx = -INFINITY;
-        const uint4* kb = reinterpret_cast<const uint4*>(p.kbar16) + static_cast<size_t>(x.bh) * p.M * kCh;
-        for (int J = gtid; J < x.cand; J += 256) {
-          float dot = 0.f;
-#pragma unroll 4
-          for (int c = 0; c < kCh; ++c) {
-            const uint4 w4 = __ldg(kb + static_cast<size_t>(J) * kCh + c);
-            const uint32_t u[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dot = fmaf(qbs[8 * c + 2 * i], __uint_as_float(u[i] << 16), dot);
-              dot = fmaf(qbs[8 * c + 2 * i + 1], __uint_as_float(u[i] & 0xffff0000u), dot);
+        if (*stop_s) return false;
+        x = make_unit(u, p);
+        if (!p.dense) {
+          // mark the listed blocks (A2 skips them), cache the list, validate it
+          const int nw = (x.cand + 31) / 32;
+          for (int i = gtid; i < nw; i += 256) bitmap[i] = 0u;
+          named_barrier_sync(1, 256);
+          bool bad = x.bad;
+          for (int i = gtid; i < x.nsel; i += 256) {
+            const int J = __ldg(p.col_idx + x.rp + i);
+            if (i < kColCache) cols[i] = J;
+            if (J < 0 || J >= x.cand) {
+              bad = true;
+            } else {
+              const uint32_t bit = 1u << (J & 31);
+              if (atomicOr(&bitmap[J >> 5], bit) & bit) bad = true;
             }
           }
-          mx = fmaxf(mx, dot);
+          if (bad) record_status(p.status, kStatusCsr);
+          named_barrier_sync(1, 256);
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) red[1024 + gwarp] = mx;
-        named_barrier_sync(1, 256);
-        float m8 = red[1024];
-#pragma unroll
-        for (int wv = 1; wv < 8; ++wv) m8 = fmaxf(m8, red[1024 + wv]);
-        c2 = m8 * p.scale_log2 + 6.0f;
-      }
-      const float bias = -c2;
+  #pragma unroll
+        for (int q = 0; q < 64; ++q) lsum[q] = 0.f;
+        // Stabiliser of the whole query block (log2 units): c2 = max over the
+        // candidate blocks of qbar_I . kbar_J / sqrt(d) * log2(e) + log2(64),
+        // with qbar_I the mean of the block's queries.  Any constant within a
+        // few tens of the rows' largest logits keeps every term in range; rows
+        // whose sum still leaves [2^-60, 2^60] are recomputed by the fixup.
+        if (p.row_max) {
+          // the router's largest block score of this row, qbar_I . kbar_J / sqrt(d)
+          c2 = __ldg(p.row_max + x.row) * 1.4426950408889634f + 6.0f;
+        } else {
+          constexpr int kCh = D / 8;             // 16-byte chunks of a row
+          constexpr int kGr = 256 / kCh;         // row groups
+          const int ch = gtid % kCh, gr = gtid / kCh;
+          const uint4* qrow = reinterpret_cast<const uint4*>(p.q) + (static_cast<size_t>(x.row) * 64) * kCh + ch;
+          float part[8];
+  #pragma unroll
+          for (int i = 0; i < 8; ++i) part[i] = 0.f;
+  #pragma unroll
+          for (int r = gr; r < 64; r += kGr) {
+            const uint4 w4 = __ldg(qrow + static_cast<size_t>(r) * kCh);
+            const uint32_t u[4] = {w4.x, w4.y, w4.z, w4.w};
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              part[2 * i] += __uint_as_float(u[i] << 16);
+              part[2 * i + 1] += __uint_as_float(u[i] & 0xffff0000u);
+            }
+          }
+  #pragma unroll
+          for (int o = kCh; o < 32; o <<= 1)
+  #pragma unroll
+            for (int i = 0; i < 8; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
+          if (lane < kCh) {
+  #pragma unroll
+            for (int i = 0; i < 8; ++i) red[gwarp * 64 * 2 + ch * 8 + i] = part[i];  // [8 warps][<=128]
+          }
+          named_barrier_sync(1, 256);
+          if (gtid < D) {
+            float sum = 0.f;
+  #pragma unroll
+            for (int wv = 0; wv < 8; ++wv) sum += red[wv * 128 + gtid];
+            qbs[gtid] = sum * (1.0f / 64.0f);
+          }
+          named_barrier_sync(1, 256);
+          float mx = -INFINITY;
+          const uint4* kb = reinterpret_cast<const uint4*>(p.kbar16) + static_cast<size_t>(x.bh) * p.M * kCh;
+          for (int J = gtid; J < x.cand; J += 256) {
+            float dot = 0.f;
+  #pragma unroll 4
+            for (int c = 0; c < kCh; ++c) {
+              const uint4 w4 = __ldg(kb + static_cast<size_t>(J) * kCh + c);
+              const uint32_t u[4] = {w4.x, w4.y, w4.z, w4.w};
+  #pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                dot = fmaf(qbs[8 * c + 2 * i], __uint_as_float(u[i] << 16), dot);
+                dot = fmaf(qbs[8 * c + 2 * i + 1], __uint_as_float(u[i] & 0xffff0000u), dot);
+              }
+            }
+            mx = fmaxf(mx, dot);
+          }
+  #pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          if (lane == 0) red[1024 + gwarp] = mx;
+          named_barrier_sync(1, 256);
+          float m8 = red[1024];
+  #pragma unroll
+          for (int wv = 1; wv < 8; ++wv) m8 = fmaxf(m8, red[1024 + wv]);
+          c2 = m8 * p.scale_log2 + 6.0f;
+        }
+        bias = -c2;
+        return true;
+    };
+    bool go = static_cast<int>(blockIdx.x) < p.units && prologue(blockIdx.x);
+    for (int u = blockIdx.x; go; u += gridDim.x, ++ul) {
 
       // ---- A2 (unlisted pooled blocks) and E (listed blocks) tiles
       for (int t = 0; t < x.ntiles; ++t, ++sc) {
@@ -646,6 +655,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (gtid == 0) bulk_wait_read0();  // the previous unit's store has read the staging tile
       named_barrier_sync(1, 256);
+      const int row_done = x.row;
+      // the next unit's setup overlaps the wait for this unit's last GEMM2
+      go = u + static_cast<int>(gridDim.x) < p.units && prologue(u + gridDim.x);
       const int ob = ul & 1;
       mbar_wait(&o_full[ob], (ul >> 1) & 1, abort_flag, p.status);
       tc_fence_after();
@@ -664,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_shared();
       named_barrier_sync(1, 256);
       if (gtid == 0) {
-        bulk_store(p.out + static_cast<size_t>(x.row) * 64 * D, sOut, C::kOutBytes);
+        bulk_store(p.out + static_cast<size_t>(row_done) * 64 * D, sOut, C::kOutBytes);
         bulk_commit();
         if (*unit_flag) {
           const int slot = atomicAdd(p.fixup_count, 1);
