@@ -100,10 +100,18 @@ struct Unit {
   bool bad;  // row_ptr entries out of range
 };
 
-__device__ __forceinline__ Unit make_unit(int u, const Params& p) {
+// Block-list row of work unit u: head-major, largest I first inside a head
+// (concurrent CTAs share one head's K/V in L2, and long causal rows are
+// scheduled first).
+__device__ __forceinline__ int unit_row(int u, const Params& p) {
+  const int bh = u / p.M;
+  return bh * p.M + p.M - 1 - (u - bh * p.M);
+}
+
+// Unit u given its row_ptr pair (a, b) = row_ptr[row], row_ptr[row + 1]
+// (ignored in dense mode).
+__device__ __forceinline__ Unit make_unit_with(int u, const Params& p, int a, int b) {
   Unit x;
-  // head-major, largest I first inside a head: concurrent CTAs share one
-  // head's K/V in L2, and long causal rows are scheduled first
   x.bh = u / p.M;
   x.I = p.M - 1 - (u - x.bh * p.M);
   x.row = x.bh * p.M + x.I;
@@ -114,7 +122,6 @@ __device__ __forceinline__ Unit make_unit(int u, const Params& p) {
     x.rp = 0;
     x.nsel = x.cand;
   } else {
-    const int a = __ldg(p.row_ptr + x.row), b = __ldg(p.row_ptr + x.row + 1);
     if (a < 0 || b < a || static_cast<long long>(b) > p.col_cap || b - a > x.cand) {
       x.bad = true;
       x.rp = 0;
@@ -131,6 +138,12 @@ __device__ __forceinline__ Unit make_unit(int u, const Params& p) {
   x.n_e = ne;
   x.ntiles = x.n_a2 + x.n_e;
   return x;
+}
+
+__device__ __forceinline__ Unit make_unit(int u, const Params& p) {
+  if (p.dense) return make_unit_with(u, p, 0, 0);
+  const int row = unit_row(u, p);
+  return make_unit_with(u, p, __ldg(p.row_ptr + row), __ldg(p.row_ptr + row + 1));
 }
 
 // tile t of a unit: pooled (A2, unlisted blocks) or exact (E, listed
@@ -181,6 +194,36 @@ __device__ __forceinline__ void group_reduce64(float (&v)[64], float* red, float
     out[gtid] = r;
   }
   named_barrier_sync(1, 256);
+}
+
+// The same column sum with one barrier: thread gtid < 64 gets out[gtid] as
+// the return value (the others get 0).  `red` must not be rewritten before
+// the group's next barrier.
+__device__ __forceinline__ float group_sum64(float (&v)[64], float* red, int lane, int gwarp, int gtid) {
+#pragma unroll
+  for (int step = 0; step < 5; ++step) {
+    const int o = 16 >> step;
+    const int half = 32 >> step;
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  const int col = ((lane & 16) ? 32 : 0) + ((lane & 8) ? 16 : 0) + ((lane & 4) ? 8 : 0) +
+                  ((lane & 2) ? 4 : 0) + ((lane & 1) ? 2 : 0);
+  red[gwarp * 64 + col] = v[0];
+  red[gwarp * 64 + col + 1] = v[1];
+  named_barrier_sync(1, 256);
+  float r = 0.f;
+  if (gtid < 64) {
+    r = red[gtid];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) r += red[w * 64 + gtid];
+  }
+  return r;
 }
 
 template <int N>
@@ -481,20 +524,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     int ul = 0;
     Unit x;
     float bias = 0.f;
-    // Start of a unit: the group-consistent stop decision, the unit's block
-    // list (bitmap of listed blocks for the pooled tiles, cached list) and
-    // its stabiliser.  Returns false when the kernel is stopping.
-    auto prologue = [&](int u) -> bool {
-        named_barrier_sync(1, 256);
-        if (gtid == 0) *stop_s = *abort_flag;
-        named_barrier_sync(1, 256);
-        if (*stop_s) return false;
-        x = make_unit(u, p);
+    // Start of a unit, after the group-consistent stop decision and the
+    // clearing of the listed-block bitmap (both done under the group barrier
+    // that precedes this): the unit's block list (bitmap of listed blocks for
+    // the pooled tiles, cached list) and its stabiliser.  (a, b) is the
+    // unit's row_ptr pair and rmax its router row maximum, loaded by the
+    // caller ahead of time.
+    auto prologue = [&](int u, int a, int b, float rmax) {
+        x = make_unit_with(u, p, a, b);
         if (!p.dense) {
           // mark the listed blocks (A2 skips them), cache the list, validate it
-          const int nw = (x.cand + 31) / 32;
-          for (int i = gtid; i < nw; i += 256) bitmap[i] = 0u;
-          named_barrier_sync(1, 256);
           bool bad = x.bad;
           for (int i = gtid; i < x.nsel; i += 256) {
             const int J = __ldg(p.col_idx + x.rp + i);
@@ -518,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // whose sum still leaves [2^-60, 2^60] are recomputed by the fixup.
         if (p.row_max) {
           // the router's largest block score of this row, qbar_I . kbar_J / sqrt(d)
-          c2 = __ldg(p.row_max + x.row) * 1.4426950408889634f + 6.0f;
+          c2 = rmax * 1.4426950408889634f + 6.0f;
         } else {
           constexpr int kCh = D / 8;             // 16-byte chunks of a row
           constexpr int kGr = 256 / kCh;         // row groups
@@ -579,9 +618,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           c2 = m8 * p.scale_log2 + 6.0f;
         }
         bias = -c2;
-        return true;
     };
-    bool go = static_cast<int>(blockIdx.x) < p.units && prologue(blockIdx.x);
+    // a unit's row_ptr pair and row maximum
+    int na = 0, nb = 0;
+    float nrmax = 0.f;
+    auto load_next = [&](int un) {
+      if (un >= p.units) return;
+      const int row = unit_row(un, p);
+      if (!p.dense) {
+        na = __ldg(p.row_ptr + row);
+        nb = __ldg(p.row_ptr + row + 1);
+      }
+      if (p.row_max) nrmax = __ldg(p.row_max + row);
+    };
+    const int nw_all = (p.M + 31) / 32;  // bitmap words of the widest candidate range
+    bool go = static_cast<int>(blockIdx.x) < p.units;
+    if (go) {
+      load_next(blockIdx.x);
+      if (gtid == 0) *stop_s = *abort_flag;
+      for (int i = gtid; i < nw_all; i += 256) bitmap[i] = 0u;
+      named_barrier_sync(1, 256);
+      go = !*stop_s;
+      if (go) prologue(blockIdx.x, na, nb, nrmax);
+    }
     for (int u = blockIdx.x; go; u += gridDim.x, ++ul) {
 
       // ---- A2 (unlisted pooled blocks) and E (listed blocks) tiles
@@ -645,19 +704,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // ---------------------------------------------------------- epilogue
-      group_reduce64<false>(lsum, red, lsh, lane, gwarp, gtid);
+      const float l = group_sum64(lsum, red, lane, gwarp, gtid);
       if (gtid < 64) {
-        const float l = lsh[gtid];
         const bool good = l >= 0x1p-60f && l <= 0x1p60f;  // false for NaN
         invl[gtid] = good ? 1.0f / l : 0.f;
         if (!good) *unit_flag = 1;
         if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + gtid] = (c2 + __log2f(l)) * kLn2;
       }
-      if (gtid == 0) bulk_wait_read0();  // the previous unit's store has read the staging tile
+      const bool more = u + static_cast<int>(gridDim.x) < p.units;
+      if (gtid == 0) {
+        bulk_wait_read0();  // the previous unit's store has read the staging tile
+        *stop_s = *abort_flag;
+      }
+      if (more && !p.dense)
+        for (int i = gtid; i < nw_all; i += 256) bitmap[i] = 0u;
       named_barrier_sync(1, 256);
       const int row_done = x.row;
       // the next unit's setup overlaps the wait for this unit's last GEMM2
-      go = u + static_cast<int>(gridDim.x) < p.units && prologue(u + gridDim.x);
+      go = more && !*stop_s;
+      if (go) {
+        load_next(u + gridDim.x);
+        prologue(u + gridDim.x, na, nb, nrmax);
+      }
       const int ob = ul & 1;
       mbar_wait(&o_full[ob], (ul >> 1) & 1, abort_flag, p.status);
       tc_fence_after();
