@@ -205,6 +205,9 @@ class Step:
         qbar, kbar, vsum = self.stats
         if self.mode == "topk":
             psa.psa_route_topk(qbar, kbar, self.param, self.causal, out=self.csr, stream=s)
+        elif self.mode == "thresh_prob":
+            psa.psa_route_thresh_prob(qbar, kbar, self.param, self.causal, self.keep_first, ws=self.ws,
+                                      out=self.csr, stream=s)
         else:
             psa.psa_route_thresh(qbar, kbar, self.param, self.causal, self.keep_first, ws=self.ws,
                                  out=self.csr, stream=s)
@@ -465,7 +468,8 @@ def oracle_step_time(name, param, budget_s):
         if mode == "topk":
             rp, ci = O.route_topk(s[b:b + 1, h:h + 1], param, causal)
         else:
-            rp, ci = O.route_thresh(s[b:b + 1, h:h + 1], param, causal, w["keep_first"])
+            route = O.route_thresh_prob if mode == "thresh_prob" else O.route_thresh
+            rp, ci = route(s[b:b + 1, h:h + 1], param, causal, w["keep_first"])
         t_route += time.perf_counter() - t1
         heads += 1
         for I in rng.permutation(M):

@@ -103,6 +103,35 @@ long long causal_prefix(long long I, long long k0) {
 
 }  // namespace
 
+namespace {
+
+// Shared by both threshold routers: thr_I = a_mul * max_J s_IJ + a_add.
+int route_thresh_common(const float* qbar, const float* kbar, int B, int H, int M, int d, float a_mul, float a_add,
+                        int causal, int keep_first, int* row_ptr, int* col_idx, size_t capacity, int* nnz_out,
+                        float* row_max, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!qbar || !kbar || !row_ptr || !col_idx || !nnz_out || !workspace) return PSA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(row_max) & 3u) return PSA_ERR_ARG;
+  if (M <= 0) return PSA_ERR_ARG;
+  if (M > kMaxBlocks) return PSA_ERR_UNSUPPORTED;
+  int s = check_shape(B, H, M * kBlock, d, kBlock);
+  if (s != PSA_OK) return s;
+  if ((causal != 0 && causal != 1) || (keep_first != 0 && keep_first != 1)) return PSA_ERR_ARG;
+  if (!aligned16(qbar) || !aligned16(kbar) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PSA_ERR_ARG;
+  const long long bh = static_cast<long long>(B) * H;
+  const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
+  if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
+  if ((s = check_device()) != PSA_OK) return s;
+  const long long cap = capacity > static_cast<size_t>(INT_MAX) ? INT_MAX : static_cast<long long>(capacity);
+  char* ws = static_cast<char*>(workspace);
+  return cuda_status(psa::launch_route_thresh(qbar, kbar, static_cast<int>(bh), M, d, a_mul, a_add, causal,
+                                              keep_first, row_ptr, col_idx, cap, nnz_out,
+                                              reinterpret_cast<int*>(ws + L.row_count),
+                                              reinterpret_cast<uint32_t*>(ws + L.row_bits), row_max,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* psa_status_string(int status) {
@@ -173,26 +202,18 @@ int psa_route_topk(const float* qbar, const float* kbar, int B, int H, int M, in
 int psa_route_thresh(const float* qbar, const float* kbar, int B, int H, int M, int d, float alpha, int causal,
                      int keep_first, int* row_ptr, int* col_idx, size_t capacity, int* nnz_out, float* row_max,
                      void* workspace, size_t workspace_bytes, void* stream) {
-  if (!qbar || !kbar || !row_ptr || !col_idx || !nnz_out || !workspace) return PSA_ERR_ARG;
-  if (reinterpret_cast<uintptr_t>(row_max) & 3u) return PSA_ERR_ARG;
-  if (M <= 0) return PSA_ERR_ARG;
-  if (M > kMaxBlocks) return PSA_ERR_UNSUPPORTED;
-  int s = check_shape(B, H, M * kBlock, d, kBlock);
-  if (s != PSA_OK) return s;
   if (!std::isfinite(alpha)) return PSA_ERR_ARG;
-  if ((causal != 0 && causal != 1) || (keep_first != 0 && keep_first != 1)) return PSA_ERR_ARG;
-  if (!aligned16(qbar) || !aligned16(kbar) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PSA_ERR_ARG;
-  const long long bh = static_cast<long long>(B) * H;
-  const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
-  if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
-  if ((s = check_device()) != PSA_OK) return s;
-  const long long cap = capacity > static_cast<size_t>(INT_MAX) ? INT_MAX : static_cast<long long>(capacity);
-  char* ws = static_cast<char*>(workspace);
-  return cuda_status(psa::launch_route_thresh(qbar, kbar, static_cast<int>(bh), M, d, alpha, causal, keep_first,
-                                              row_ptr, col_idx, cap, nnz_out,
-                                              reinterpret_cast<int*>(ws + L.row_count),
-                                              reinterpret_cast<uint32_t*>(ws + L.row_bits), row_max,
-                                              static_cast<cudaStream_t>(stream)));
+  return route_thresh_common(qbar, kbar, B, H, M, d, alpha, 0.0f, causal, keep_first, row_ptr, col_idx, capacity,
+                             nnz_out, row_max, workspace, workspace_bytes, stream);
+}
+
+int psa_route_thresh_prob(const float* qbar, const float* kbar, int B, int H, int M, int d, float alpha,
+                          int causal, int keep_first, int* row_ptr, int* col_idx, size_t capacity, int* nnz_out,
+                          float* row_max, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!(alpha > 0.0f) || !std::isfinite(alpha)) return PSA_ERR_ARG;
+  const float log_alpha = static_cast<float>(std::log(static_cast<double>(alpha)));
+  return route_thresh_common(qbar, kbar, B, H, M, d, 1.0f, log_alpha, causal, keep_first, row_ptr, col_idx,
+                             capacity, nnz_out, row_max, workspace, workspace_bytes, stream);
 }
 
 int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar, const float* vsum,

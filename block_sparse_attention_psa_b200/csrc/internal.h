@@ -37,8 +37,9 @@ cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long
 cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int M, int d, int k0, int causal,
                               int* row_ptr, int* col_idx, long long total, int* nnz_out, float* row_max,
                               cudaStream_t st);
-cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, int M, int d, float alpha,
-                                int causal, int keep_first, int* row_ptr, int* col_idx, long long capacity,
+// threshold thr_I = a_mul * max_J s_IJ + a_add (one fma)
+cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, int M, int d, float a_mul,
+                                float a_add, int causal, int keep_first, int* row_ptr, int* col_idx, long long capacity,
                                 int* nnz_out, int* row_count, uint32_t* row_bits, float* row_max,
                                 cudaStream_t st);
 

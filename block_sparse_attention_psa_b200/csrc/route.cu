@@ -207,7 +207,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 template <int R, int D>
 __global__ void __launch_bounds__(256) route_thresh_kernel(const float* __restrict__ qbar,
                                                            const float* __restrict__ kbar, int M,
-                                                           float tau, float alpha, int causal, int keep_first,
+                                                           float tau, float a_mul, float a_add, int causal,
+                                                           int keep_first,
                                                            int* __restrict__ row_count,
                                                            uint32_t* __restrict__ row_bits,
                                                            float* __restrict__ row_max) {
@@ -231,7 +232,9 @@ __global__ void __launch_bounds__(256) route_thresh_kernel(const float* __restri
   for (int J = lane; J < cand; J += 32) m = fmaxf(m, s[J]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  const float thr = alpha * m;
+  // logit rule: alpha * max (a_mul = alpha, a_add = 0, the product exactly as
+  // alpha * m); probability rule: max + ln(alpha) (a_mul = 1, a_add = ln alpha)
+  const float thr = fmaf(a_mul, m, a_add);
   if (row_max && lane == 0) row_max[row] = m;
   const int nw = (M + 31) / 32;
   uint32_t* bits = row_bits + row * nw;
@@ -380,8 +383,8 @@ cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int 
   return cudaGetLastError();
 }
 
-cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, int M, int d, float alpha,
-                                int causal, int keep_first, int* row_ptr, int* col_idx, long long capacity,
+cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, int M, int d, float a_mul,
+                                float a_add, int causal, int keep_first, int* row_ptr, int* col_idx, long long capacity,
                                 int* nnz_out, int* row_count, uint32_t* row_bits, float* row_max,
                                 cudaStream_t st) {
   const int R = rows_per_cta(M, d);
@@ -393,11 +396,11 @@ cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, in
   case RR:                                                                                             \
     if (d == 128) {                                                                                    \
       if ((e = set_smem(route_thresh_kernel<RR, 128>, smem)) != cudaSuccess) return e;                 \
-      route_thresh_kernel<RR, 128><<<grid, 256, smem, st>>>(qbar, kbar, M, tau, alpha, causal,         \
+      route_thresh_kernel<RR, 128><<<grid, 256, smem, st>>>(qbar, kbar, M, tau, a_mul, a_add, causal,  \
                                                              keep_first, row_count, row_bits, row_max); \
     } else {                                                                                           \
       if ((e = set_smem(route_thresh_kernel<RR, 64>, smem)) != cudaSuccess) return e;                  \
-      route_thresh_kernel<RR, 64><<<grid, 256, smem, st>>>(qbar, kbar, M, tau, alpha, causal,          \
+      route_thresh_kernel<RR, 64><<<grid, 256, smem, st>>>(qbar, kbar, M, tau, a_mul, a_add, causal,   \
                                                             keep_first, row_count, row_bits, row_max);  \
     }                                                                                                  \
     break;

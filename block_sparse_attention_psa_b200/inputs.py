@@ -44,6 +44,12 @@ WORKLOADS = {
     "dit_video_n32k_thresh": dict(B=1, H=12, N=32768, d=128, gen="clustered",
                                   causal=False, routing=("thresh", 0.5),
                                   keep_first=False),
+    # same tensors, threshold alpha = 0.5 read in the probability domain: keep
+    # blocks whose softmax weight is at least half the row's largest
+    # (s >= max + ln 0.5)
+    "dit_video_n32k_thresh_prob": dict(B=1, H=12, N=32768, d=128, gen="clustered",
+                                       causal=False, routing=("thresh_prob", 0.5),
+                                       keep_first=False),
     # long causal prefill, threshold 0.5, block 0 and diagonal always kept
     "long_causal_n128k": dict(B=1, H=8, N=131072, d=128, gen="clustered_slash",
                               causal=True, routing=("thresh", 0.5), keep_first=True),

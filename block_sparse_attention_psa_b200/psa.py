@@ -30,7 +30,7 @@ PSA_ERR_DEVICE = 8
 
 EXPORTS = ("psa_status_string", "psa_version", "psa_workspace_size", "psa_route_capacity", "psa_pool",
            "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense", "psa_read_status",
-           "psa_attn_noalloc")
+           "psa_attn_noalloc", "psa_route_thresh_prob")
 
 _lib = None
 
@@ -51,6 +51,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "psa_pool": (I, [P, P, P, I, I, I, I, I, P, P, P, P]),
         "psa_route_topk": (I, [P, P, I, I, I, I, F, I, P, P, Z, P, P, P]),
         "psa_route_thresh": (I, [P, P, I, I, I, I, F, I, I, P, P, Z, P, P, P, Z, P]),
+        "psa_route_thresh_prob": (I, [P, P, I, I, I, I, F, I, I, P, P, Z, P, P, P, Z, P]),
         "psa_attn": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, Z, P]),
         "psa_dense": (I, [P, P, P, I, I, I, I, I, P, P, P, Z, P]),
         "psa_read_status": (I, [P, ctypes.POINTER(I), P]),
@@ -171,6 +172,22 @@ def psa_route_thresh(qbar, kbar, alpha: float, causal: bool = False, keep_first:
     return row_ptr, col_idx, nnz, row_max
 
 
+def psa_route_thresh_prob(qbar, kbar, alpha: float, causal: bool = False, keep_first: bool = False,
+                          ws=None, capacity: int | None = None, out=None, stream=None):
+    """Threshold routing in the probability domain: keep J iff
+    s_IJ >= max_J s_IJ + ln(alpha).  Returns (row_ptr, col_idx, nnz, row_max)."""
+    B, H, M, d = (int(x) for x in qbar.shape)
+    if ws is None:
+        ws = workspace(B, H, M * 64, d, qbar.device)
+    if out is None:
+        out = _route_out(B, H, M, causal, capacity, qbar.device)
+    row_ptr, col_idx, nnz, row_max = out
+    _check("psa_route_thresh_prob", lib().psa_route_thresh_prob(
+        _ptr(qbar), _ptr(kbar), B, H, M, d, float(alpha), int(causal), int(keep_first), _ptr(row_ptr),
+        _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(row_max), _ptr(ws), ws.numel(), _stream(stream)))
+    return row_ptr, col_idx, nnz, row_max
+
+
 def psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_size: int = 64,
              ws=None, out=None, lse=None, want_lse: bool = False, row_max=None, stream=None):
     """Returns out (bf16 [B,H,N,d]) and, if requested, lse (float32 [B,H,N]).
@@ -243,7 +260,9 @@ def psa_forward(q, k, v, mode: str = "topk", density: float = 0.15, alpha: float
         csr = psa_route_topk(qbar, kbar, density, causal, stream=stream)
     elif mode == "thresh":
         csr = psa_route_thresh(qbar, kbar, alpha, causal, keep_first, ws=ws, stream=stream)
+    elif mode == "thresh_prob":
+        csr = psa_route_thresh_prob(qbar, kbar, alpha, causal, keep_first, ws=ws, stream=stream)
     else:
-        raise ValueError("mode must be 'topk' or 'thresh'")
+        raise ValueError("mode must be 'topk', 'thresh' or 'thresh_prob'")
     out = psa_attn(q, k, v, kbar, vsum, csr[0], csr[1], causal, ws=ws, row_max=csr[3], stream=stream)
     return out, csr

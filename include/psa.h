@@ -133,6 +133,24 @@ PSA_API int psa_route_thresh(const float* qbar, const float* kbar,
                      size_t workspace_bytes, void* stream);
 
 /*
+ * a4, probability reading. The same max-based rule with the block attention
+ * score read as the softmax of the row's block scores [FlashPrefill summary,
+ * 2.b "Max-based dynamic thresholding"; the summary does not say which
+ * score it means]: keep J iff p_IJ >= alpha * max_J p_IJ with p_IJ
+ * proportional to e^{s_IJ}, i.e. s_IJ >= max_J s_IJ + ln(alpha) (float32,
+ * ln(alpha) rounded to float32), plus the diagonal block I, plus block 0
+ * when keep_first.  alpha must be positive and finite (alpha >= 1 keeps the
+ * row maximum and the forced blocks only).  Outputs, workspace, capacity
+ * and errors as psa_route_thresh; row_max (nullable) is still the row
+ * maximum of s_IJ.
+ */
+PSA_API int psa_route_thresh_prob(const float* qbar, const float* kbar,
+                          int B, int H, int M, int d, float alpha, int causal,
+                          int keep_first, int* row_ptr, int* col_idx, size_t capacity,
+                          int* nnz_out, float* row_max, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
  * a5 - a7. Exact attention on the listed blocks plus the 0th-order term of
  * every other candidate, in one softmax [PISA summary, routing table and
  * "Why approximating unselected blocks keeps softmax intact"; FlashPrefill

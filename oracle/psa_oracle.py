@@ -48,6 +48,9 @@ Readings where the pages are silent (each is listed in the design doc):
   best of the blocks J < I;
 * threshold: keep J iff s_IJ >= alpha * max_J' s_IJ' over the candidates,
   plus the diagonal block I, plus block 0 when ``keep_first``;
+* threshold, probability reading (``route_thresh_prob``): the "attention
+  score" of the rule taken as the softmax of the row's block scores, which
+  makes it s_IJ >= max_J' s_IJ' + ln(alpha), same forced blocks;
 * causal: candidates are J <= I; inside the diagonal block key j is visible to
   query i iff j <= i; blocks J > I contribute nothing, not even their 0th
   order term; the diagonal block never gets a 0th-order term (its pooled key
@@ -192,6 +195,34 @@ def route_thresh(s, alpha: float, causal: bool, keep_first: bool):
                 thresh = alpha * vals.max()
                 keep = vals >= thresh
                 keep[min(I, n_cand - 1)] = True   # diagonal block (I < M always)
+                if keep_first:
+                    keep[0] = True
+                lists.append(np.nonzero(keep)[0])
+    return _to_csr(lists)
+
+
+def route_thresh_prob(s, alpha: float, causal: bool, keep_first: bool):
+    """The same max-based rule read in the probability domain (FlashPrefill
+    summary, 2.b "Max-based dynamic thresholding", with the block attention
+    score taken as the softmax of the row's block scores): keep J iff
+    p_IJ >= alpha * max_J p_IJ, where p_IJ = e^{s_IJ} / sum over the candidates.
+    The normaliser cancels in the ratio, so this is s_IJ >= max_J s_IJ + ln(alpha),
+    evaluated here in that form; plus the diagonal block I, plus block 0 when
+    ``keep_first``.  alpha > 0.  Lists ascending."""
+    s = _f64(s)
+    B, H, M, _ = s.shape
+    alpha = float(np.float32(alpha))
+    if not alpha > 0:
+        raise ValueError("alpha must be positive")
+    log_alpha = math.log(alpha)
+    lists = []
+    for b in range(B):
+        for h in range(H):
+            for I in range(M):
+                n_cand = candidate_count(I, M, causal)
+                vals = s[b, h, I, :n_cand]
+                keep = vals >= vals.max() + log_alpha
+                keep[min(I, n_cand - 1)] = True
                 if keep_first:
                     keep[0] = True
                 lists.append(np.nonzero(keep)[0])

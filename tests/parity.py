@@ -13,6 +13,8 @@ Rules (fixed before any kernel was written):
 
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import torch
 
@@ -39,6 +41,8 @@ def run_gpu(q, k, v, mode, param, causal=False, keep_first=False, want_lse=True,
     qbar, kbar, vsum = psa.psa_pool(dq, dk, dv)
     if mode == "topk":
         row_ptr, col_idx, nnz, row_max = psa.psa_route_topk(qbar, kbar, param, causal)
+    elif mode == "thresh_prob":
+        row_ptr, col_idx, nnz, row_max = psa.psa_route_thresh_prob(qbar, kbar, param, causal, keep_first, ws=ws)
     else:
         row_ptr, col_idx, nnz, row_max = psa.psa_route_thresh(qbar, kbar, param, causal, keep_first, ws=ws)
     out, lse = psa.psa_attn(dq, dk, dv, kbar, vsum, row_ptr, col_idx, causal, ws=ws, want_lse=True,
@@ -76,6 +80,8 @@ def check_routing(g, s, mode, param, causal, keep_first=False):
     B, H, M, _ = s.shape
     if mode == "topk":
         rp_ref, ci_ref = O.route_topk(s, param, causal)
+    elif mode == "thresh_prob":
+        rp_ref, ci_ref = O.route_thresh_prob(s, param, causal, keep_first)
     else:
         rp_ref, ci_ref = O.route_thresh(s, param, causal, keep_first)
     rp, ci = g["row_ptr"], g["col_idx"]
@@ -106,7 +112,10 @@ def check_routing(g, s, mode, param, causal, keep_first=False):
                     if causal:
                         assert I in got, f"row {r}: causal diagonal missing"
                 else:
-                    ref = param * row.max()
+                    if mode == "thresh_prob":
+                        ref = row.max() + math.log(float(np.float32(param)))
+                    else:
+                        ref = param * row.max()
                     assert I in got, f"row {r}: diagonal missing"
                     if keep_first:
                         assert 0 in got, f"row {r}: block 0 missing"

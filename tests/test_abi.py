@@ -83,6 +83,12 @@ def test_host_validation_rejects_bad_arguments():
                       None, ctypes.c_void_p((1 << 20) + 16), ws, S) == psa.PSA_ERR_ARG
     assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, None, 1, 1, 64 * 16385, 64, 64, 0, FAKE,
                       None, FAKE, 1 << 40, S) == psa.PSA_ERR_UNSUPPORTED
+    # probability-domain threshold: alpha must be positive and finite
+    for bad_alpha in (0.0, -0.5, float("nan"), float("inf")):
+        assert L.psa_route_thresh_prob(FAKE, FAKE, 1, 2, 16, 64, bad_alpha, 0, 0, FAKE, FAKE, 1 << 20, FAKE, None,
+                                       FAKE, 1 << 30, S) == psa.PSA_ERR_ARG
+    assert L.psa_route_thresh_prob(FAKE, FAKE, 1, 2, 16, 64, 0.5, 0, 0, FAKE, FAKE, 1 << 20, FAKE, None, FAKE, 16,
+                                   S) == psa.PSA_ERR_CAPACITY
     # misaligned row maxima (routers' output, attention's input)
     odd = ctypes.c_void_p((1 << 20) + 2)
     assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 1 << 20, FAKE, odd, S) \

@@ -46,6 +46,13 @@ def test_clustered_threshold(d, causal, keep_first):
     _full_check(q, k, v, "thresh", 0.5, causal, keep_first)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal,keep_first", [(False, False), (True, True)])
+def test_clustered_threshold_probability_domain(d, causal, keep_first):
+    q, k, v = make_qkv(1, 3, 45 * 64, d, "clustered_slash", seed=19)
+    _full_check(q, k, v, "thresh_prob", 0.05, causal, keep_first)
+
+
 def test_many_pooled_tiles():
     # M = 300 > 2 * 128: several pooled-key tiles per unit, ragged last tile
     q, k, v = make_qkv(1, 1, 300 * 64, 64, "clustered", seed=5)
@@ -204,6 +211,19 @@ def test_full_dit_video_topk():
 
 def test_full_dit_video_threshold():
     _full_size("dit_video_n32k_thresh")
+
+
+def test_full_dit_video_threshold_probability_domain():
+    # the DiT-video tensors with the probability-domain rule: keep blocks whose
+    # softmax weight is at least 5% of the row's largest
+    w = WORKLOADS["dit_video_n32k"]
+    q, k, v = workload_inputs("dit_video_n32k")
+    g = run_gpu(q, k, v, "thresh_prob", 0.05)
+    assert g["status"] == psa.PSA_OK
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    check_routing(g, O.block_scores(qbar, kbar), "thresh_prob", 0.05, False)
+    units = sample_units(w["B"], w["H"], w["N"] // 64, 40, seed=5, g=g)
+    check_output(g, q, k, v, kbar, vsum, False, units)
 
 
 def test_full_long_causal_threshold():

@@ -186,6 +186,48 @@ def test_threshold_bruteforce_and_limits():
             r += 1
 
 
+def test_threshold_prob_is_the_softmax_ratio_rule():
+    # probability reading: p_IJ >= alpha * max p, with p the softmax of the
+    # row's candidate scores, written out here with the normaliser
+    rng = np.random.default_rng(17)
+    s = 3.0 * rng.standard_normal((1, 2, 9, 9))
+    alpha = 0.25
+    for causal in (False, True):
+        for kf in (False, True):
+            rp, ci = O.route_thresh_prob(s, alpha, causal, kf)
+            r = 0
+            for h in range(2):
+                for I in range(9):
+                    n = I + 1 if causal else 9
+                    e = np.exp(s[0, h, I, :n] - s[0, h, I, :n].max())
+                    p = e / e.sum()
+                    want = [J for J in range(n) if p[J] >= np.float32(alpha) * p.max()
+                            or J == I or (kf and J == 0)]
+                    assert list(ci[rp[r]:rp[r + 1]]) == want
+                    r += 1
+
+
+def test_threshold_prob_limits_and_shift_invariance():
+    rng = np.random.default_rng(18)
+    s = rng.standard_normal((1, 1, 8, 8))
+    # alpha = 1 keeps the row's best block (plus the forced ones); a tiny alpha keeps all
+    rp, ci = O.route_thresh_prob(s, 1.0, False, False)
+    for I in range(8):
+        assert list(ci[rp[I]:rp[I + 1]]) == sorted({int(np.argmax(s[0, 0, I])), I})
+    rp, ci = O.route_thresh_prob(s, 1e-30, True, False)
+    for I in range(8):
+        assert list(ci[rp[I]:rp[I + 1]]) == list(range(I + 1))
+    # only score differences matter: a per-row shift keeps every list, while the
+    # logit-domain rule (alpha times the max) moves
+    shift = 5.0 * rng.standard_normal((1, 1, 8, 1))
+    a = O.route_thresh_prob(s, 0.3, False, False)
+    b = O.route_thresh_prob(s + shift, 0.3, False, False)
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+    c = O.route_thresh(s, 0.3, False, False)
+    d = O.route_thresh(s + shift, 0.3, False, False)
+    assert not all(np.array_equal(x, y) for x, y in zip(c, d))
+
+
 def test_routing_invariant_to_positive_query_scale():
     rng = np.random.default_rng(7)
     qbar = rng.standard_normal((1, 2, 9, 4))
