@@ -1,6 +1,7 @@
 // api.cu -- the C ABI declared in include/psa.h: argument validation on the
 // host, workspace layout, TMA descriptor encoding and kernel launches.
 #include <climits>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -66,6 +67,10 @@ int device_sm_count() {
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 1;
   return n;
 }
+
+std::atomic<int> g_stall_request{0};
+
+int take_stall_request() { return g_stall_request.exchange(0); }
 
 }  // namespace psa
 
@@ -253,6 +258,7 @@ int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, cons
   a.col_idx = col_idx;
   a.col_cap = col_capacity > static_cast<size_t>(LLONG_MAX) ? LLONG_MAX : static_cast<long long>(col_capacity);
   a.row_max = row_max;
+  a.stall = psa::take_stall_request();
   a.out = out;
   a.lse = lse;
   a.BH = static_cast<int>(bh);
@@ -307,6 +313,12 @@ int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int
   a.fixup_count = reinterpret_cast<int*>(ws) + 1;
   a.fixup_list = reinterpret_cast<int*>(ws + L.fixup_list);
   return cuda_status(psa::launch_attn(a, st));
+}
+
+int psa_test_stall_next_attn(int on) {
+  if (on != 0 && on != 1) return PSA_ERR_ARG;
+  psa::g_stall_request.store(on);
+  return PSA_OK;
 }
 
 int psa_read_status(const void* workspace, int* status, void* stream) {

@@ -88,6 +88,7 @@ struct Params {
   __nv_bfloat16* out;
   float* lse;
   int BH, M, causal, dense, units;
+  int stall;         // test hook: CTA 0 withholds its first S^T hand-off
   float scale_log2;  // log2(e) / sqrt(d)
   int* status;
   int* fixup_count;
@@ -451,7 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 1; kk < D / 16; ++kk)
             tc_mma_bf16(dt, a + (kk >> 2) * 1024 + (kk & 3) * 2, dq + (kk >> 2) * 512 + (kk & 3) * 2,
                         C::kIdesc1, 1u);
-          tc_commit(&s_full[sb]);
+          // (the failure-path test hook withholds the first hand-off of CTA 0, so
+          // the bounded waits behind it run out; nothing else changes)
+          if (!(p.stall && blockIdx.x == 0 && sc == 0)) tc_commit(&s_full[sb]);
           if (t == x.ntiles - 1) tc_commit(&q_empty[qb]);
         }
       }
@@ -873,6 +876,7 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   p.status = a.status;
   p.fixup_count = a.fixup_count;
   p.fixup_list = a.fixup_list;
+  p.stall = a.stall;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;

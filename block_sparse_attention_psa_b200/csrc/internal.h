@@ -62,8 +62,12 @@ struct AttnLaunch {
   int* status;
   int* fixup_count;
   int* fixup_list;
+  int stall;  // failure-path test hook (0 in normal use)
 };
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t st);
+
+// api.cu: one-shot flag set by psa_test_stall_next_attn, taken by the next psa_attn
+int take_stall_request();
 
 // api.cu: driver entry point for cuTensorMapEncodeTiled (resolved once)
 CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,

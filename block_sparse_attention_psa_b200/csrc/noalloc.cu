@@ -107,6 +107,7 @@ int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
   a.col_idx = col_idx;
   a.col_cap = col_capacity > static_cast<size_t>(LLONG_MAX) ? LLONG_MAX : static_cast<long long>(col_capacity);
   a.row_max = row_max;
+  a.stall = 0;
   a.out = out;
   a.lse = lse;
   a.BH = static_cast<int>(bh);

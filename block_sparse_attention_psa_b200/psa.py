@@ -30,7 +30,7 @@ PSA_ERR_DEVICE = 8
 
 EXPORTS = ("psa_status_string", "psa_version", "psa_workspace_size", "psa_route_capacity", "psa_pool",
            "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense", "psa_read_status",
-           "psa_attn_noalloc", "psa_route_thresh_prob")
+           "psa_attn_noalloc", "psa_route_thresh_prob", "psa_test_stall_next_attn")
 
 _lib = None
 
@@ -55,6 +55,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "psa_attn": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, Z, P]),
         "psa_dense": (I, [P, P, P, I, I, I, I, I, P, P, P, Z, P]),
         "psa_read_status": (I, [P, ctypes.POINTER(I), P]),
+        "psa_test_stall_next_attn": (I, [I]),
         "psa_attn_noalloc": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -238,6 +239,12 @@ def psa_attn_noalloc(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False
         _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(status),
         _stream(stream)))
     return out
+
+
+def psa_test_stall_next_attn(on: bool = True) -> None:
+    """Failure-path test hook: the next psa_attn call's kernel lets a bounded
+    wait run out and records PSA_ERR_TIMEOUT in its workspace status word."""
+    _check("psa_test_stall_next_attn", lib().psa_test_stall_next_attn(int(bool(on))))
 
 
 def psa_read_status(ws, stream=None) -> int:

@@ -219,6 +219,17 @@ PSA_API int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa
                              int causal, psa_bf16_t* out, float* lse, int* status, void* stream);
 
 /*
+ * Test hook for the failure path (the method's sources have no counterpart;
+ * never needed in normal use).  With on = 1, the next psa_attn call (only
+ * that one, in this process) launches a kernel whose first block withholds
+ * one internal hand-off, so the bounded waits behind it run out: the call
+ * itself returns PSA_OK, the kernel stops within a few seconds and records
+ * PSA_ERR_TIMEOUT in the workspace status word, and later calls run normally
+ * on the same context.  on = 0 cancels a pending request.  Errors: PSA_ERR_ARG.
+ */
+PSA_API int psa_test_stall_next_attn(int on);
+
+/*
  * Synchronises `stream`, then copies the device status word of `workspace`
  * into *status (host pointer): PSA_OK, or the first device-side error
  * recorded since the last call that reset it (psa_route_thresh, psa_attn
