@@ -4,6 +4,8 @@ Small cases run the oracle on every unit; the full-size workloads run the
 GPU exactly as ``bench.py`` launches it and compare every block list plus a
 seeded sample of query blocks."""
 
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -273,3 +275,23 @@ def test_topk_ties_go_to_smaller_blocks(causal):
         else:
             want = list(range(kk))
         assert got == want, (r, got, want)
+
+
+# ------------------------------------------------------------------ size limits
+def test_maximum_block_count():
+    # M = 16384 key blocks (N = 1,048,576 tokens), the largest the library
+    # accepts: widest bitmap and score rows, one query row per router block
+    M, d = 16384, 64
+    q, k, v = make_qkv(1, 1, M * 64, d, "clustered", seed=22)
+    g = run_gpu(q, k, v, "topk", 0.002)
+    assert g["status"] == psa.PSA_OK
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    s = O.block_scores(qbar, kbar)
+    # routing: every row against the oracle (k = ceil(fl32(0.002 * 16384)) = 33)
+    check_routing(g, s, "topk", 0.002, False)
+    check_output(g, q, k, v, kbar, vsum, False, sample_units(1, 1, M, 12, seed=6, g=g))
+    # one block more is refused on the host
+    L = psa.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.psa_pool(fake, fake, fake, 1, 1, (M + 1) * 64, d, 64, fake, fake, fake, None) == \
+        psa.PSA_ERR_UNSUPPORTED
