@@ -67,9 +67,9 @@ struct Cfg {
   static constexpr int kOffP = kOffV + kNV * kKVBytes;   // one P^T tile per softmax warpgroup
   static constexpr int kOffOut = kOffP + 2 * kPBytes;
   static constexpr int kOffMisc = kOffOut + kOutBytes;
-  // misc: 32 barriers (256 B) + tmem slot / flags (256 B) + red[8][128 + 1]
-  // f32 + qbar[128] + invl[64] + l[64] + bitmap[kMaxBlocks / 32] + cols[kColCache]
-  static constexpr int kMiscBytes = 256 + 256 + (8 * 128 + 8) * 4 + 128 * 4 + 2 * 64 * 4 + kMaxBlocks / 8 +
+  // misc: 32 barriers (256 B) + tmem slot / flags (256 B) + red[8][128] + [8]
+  // f32 + qbar[128] + invl[64] + bitmap[kMaxBlocks / 32] + cols[kColCache]
+  static constexpr int kMiscBytes = 256 + 256 + (8 * 128 + 8) * 4 + 128 * 4 + 64 * 4 + kMaxBlocks / 8 +
                                     kColCache * 4;
   static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
   // kind::f16, bf16 x bf16 -> f32.  GEMM1: M=128 keys, N=64 queries, both
@@ -163,43 +163,12 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Column reduction over the 256 softmax threads (8 warps): v[64] per thread,
-// out[q] = sum (or max) over threads of v[q].  Butterfly transpose-reduce
-// inside each warp (after it, lane L holds columns 2*rev5(L) and +1), then
-// the eight warps combine through shared memory.
-template <bool kMax>
-__device__ __forceinline__ void group_reduce64(float (&v)[64], float* red, float* out, int lane, int gwarp,
-                                               int gtid) {
-#pragma unroll
-  for (int step = 0; step < 5; ++step) {
-    const int o = 16 >> step;
-    const int half = 32 >> step;
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = upper ? v[i] : v[i + half];
-      const float keep = upper ? v[i + half] : v[i];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, o);
-      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
-    }
-  }
-  const int col = ((lane & 16) ? 32 : 0) + ((lane & 8) ? 16 : 0) + ((lane & 4) ? 8 : 0) +
-                  ((lane & 2) ? 4 : 0) + ((lane & 1) ? 2 : 0);
-  red[gwarp * 64 + col] = v[0];
-  red[gwarp * 64 + col + 1] = v[1];
-  named_barrier_sync(1, 256);
-  if (gtid < 64) {
-    float r = red[gtid];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) r = kMax ? fmaxf(r, red[w * 64 + gtid]) : r + red[w * 64 + gtid];
-    out[gtid] = r;
-  }
-  named_barrier_sync(1, 256);
-}
-
-// The same column sum with one barrier: thread gtid < 64 gets out[gtid] as
-// the return value (the others get 0).  `red` must not be rewritten before
-// the group's next barrier.
+// Column sums over the 256 softmax threads (8 warps): v[64] per thread;
+// thread gtid < 64 gets the sum over all threads of v[gtid] as the return
+// value (the others get 0).  Butterfly transpose-reduce inside each warp
+// (after it, lane L holds columns 2*rev5(L) and +1), then the eight warps
+// combine through shared memory behind one barrier; `red` must not be
+// rewritten before the group's next barrier.
 __device__ __forceinline__ float group_sum64(float (&v)[64], float* red, int lane, int gwarp, int gtid) {
 #pragma unroll
   for (int step = 0; step < 5; ++step) {
@@ -300,8 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* red = reinterpret_cast<float*>(smem + C::kOffMisc + 512);  // [8][128] + [8]
   float* qbs = red + 8 * 128 + 8;  // block mean of the unit's queries [128]
   float* invl = qbs + 128;
-  float* lsh = invl + 64;
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(lsh + 64);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(invl + 64);
   int* cols = reinterpret_cast<int*>(bitmap + kMaxBlocks / 32);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
