@@ -30,6 +30,10 @@ __device__ __forceinline__ uint16_t f2bf(float x) {
 }
 
 // NT = number of input tensors pooled (3: q, k, v; 1: k only, bf16 mean out).
+// A work item is one tensor of one block (64 rows), so a grid-stride loop
+// has 3x more, smaller items than blocks: the last wave of CTAs is then a
+// small part of the pass even when the block count is only a few times the
+// number of resident CTAs.
 template <int D, int NT>
 __global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                                                    const uint4* __restrict__ v, int nblk,
@@ -38,43 +42,38 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ q, 
   constexpr int kChunks = D / 8;           // 16-byte chunks per row
   constexpr int kGroups = 256 / kChunks;   // row groups per CTA
   constexpr int kRows = 64 / kGroups;      // rows per thread per block
-  __shared__ float red[8][NT][D];
+  __shared__ float red[8][D];
   const int c = threadIdx.x % kChunks;
   const int g = threadIdx.x / kChunks;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const uint4* src[3] = {NT == 3 ? q : k, k, v};
+  const int items = nblk * NT;
 
-  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+  for (int it = blockIdx.x; it < items; it += gridDim.x) {
+    const int blk = it / NT, t = it - blk * NT;
+    const uint4* src = NT == 1 ? k : (t == 0 ? q : (t == 1 ? k : v));
     const size_t base = static_cast<size_t>(blk) * 64 * kChunks;
-    uint4 w[NT][kRows];
+    uint4 w[kRows];
 #pragma unroll
-    for (int t = 0; t < NT; ++t)
+    for (int r = 0; r < kRows; ++r) w[r] = __ldcs(src + base + static_cast<size_t>(g + r * kGroups) * kChunks + c);
+    float acc[8];
 #pragma unroll
-      for (int r = 0; r < kRows; ++r)
-        w[t][r] = __ldcs(src[t] + base + static_cast<size_t>(g + r * kGroups) * kChunks + c);
-    float acc[NT][8];
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
+    for (int r = 0; r < kRows; ++r) add_bf16x8(acc, w[r]);
+    // lanes that hold the same chunk differ by multiples of kChunks
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[t][i] = 0.f;
+    for (int o = kChunks; o < 32; o <<= 1)
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) add_bf16x8(acc[t], w[t][r]);
-      // lanes that hold the same chunk differ by multiples of kChunks
+      for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    if (lane < kChunks) {
 #pragma unroll
-      for (int o = kChunks; o < 32; o <<= 1)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[t][i] += __shfl_xor_sync(0xffffffffu, acc[t][i], o);
-      if (lane < kChunks) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) red[warp][t][c * 8 + i] = acc[t][i];
-      }
+      for (int i = 0; i < 8; ++i) red[warp][c * 8 + i] = acc[i];
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < NT * D; e += 256) {
-      const int t = e / D, col = e % D;
+    for (int col = threadIdx.x; col < D; col += 256) {
       float s = 0.f;
 #pragma unroll
-      for (int wi = 0; wi < 8; ++wi) s += red[wi][t][col];
+      for (int wi = 0; wi < 8; ++wi) s += red[wi][col];
       const size_t o = static_cast<size_t>(blk) * D + col;
       if (NT == 3) {
         if (t == 0) qbar[o] = s * (1.0f / 64.0f);
@@ -101,9 +100,9 @@ __global__ void stats_to_bf16_kernel(const float4* __restrict__ kbar, const floa
   }
 }
 
-int pool_grid(int nblk) {
+int pool_grid(long long items) {
   const int cap = device_sm_count() * 8;
-  return nblk < cap ? nblk : cap;
+  return items < cap ? static_cast<int>(items) : cap;
 }
 
 }  // namespace
@@ -111,7 +110,7 @@ int pool_grid(int nblk) {
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int M, int d,
                         float* qbar, float* kbar, float* vsum, cudaStream_t st) {
   const int nblk = BH * M;
-  const dim3 grid(pool_grid(nblk));
+  const dim3 grid(pool_grid(3LL * nblk));
   auto* Q = reinterpret_cast<const uint4*>(q);
   auto* K = reinterpret_cast<const uint4*>(k);
   auto* V = reinterpret_cast<const uint4*>(v);
