@@ -295,3 +295,61 @@ def test_maximum_block_count():
     fake = ctypes.c_void_p(1 << 20)
     assert L.psa_pool(fake, fake, fake, 1, 1, (M + 1) * 64, d, 64, fake, fake, fake, None) == \
         psa.PSA_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ capacity and streams
+def test_threshold_truncation_keeps_a_valid_prefix():
+    # a col_idx buffer half the exact total: the exact total is still reported,
+    # rows past the capacity are cut, and the cut CSR is a valid input to attention
+    q, k, v = make_qkv(1, 2, 40 * 64, 64, "clustered", seed=23)
+    dq, dk, dv = (x.cuda() for x in (q, k, v))
+    B, H, N, d = q.shape
+    M = N // 64
+    ws = psa.workspace(B, H, N, d)
+    qbar, kbar, vsum = psa.psa_pool(dq, dk, dv)
+    rp_f, ci_f, nnz_f, _ = psa.psa_route_thresh(qbar, kbar, 0.5, ws=ws)
+    total = int(nnz_f.item())
+    cap = total // 2
+    rp_t, ci_t, nnz_t, rmax_t = psa.psa_route_thresh(qbar, kbar, 0.5, ws=ws, capacity=cap)
+    assert int(nnz_t.item()) == total
+    rp_f, rp_t = rp_f.cpu().long().numpy(), rp_t.cpu().long().numpy()
+    ci_f, ci_t = ci_f.cpu().long().numpy(), ci_t[:cap].cpu().long().numpy()
+    assert np.all(np.diff(rp_t) >= 0) and rp_t[0] == 0 and rp_t[-1] == cap
+    for r in range(B * H * M):
+        got = ci_t[rp_t[r]:rp_t[r + 1]]
+        full = ci_f[rp_f[r]:rp_f[r + 1]]
+        assert np.array_equal(got, full[:got.size]), r
+        if rp_f[r + 1] <= cap:
+            assert got.size == full.size, r
+    # attention over the cut lists
+    ci_dev = torch.tensor(ci_t if cap else [0], dtype=torch.int32, device="cuda")
+    rp_dev = torch.tensor(rp_t, dtype=torch.int32, device="cuda")
+    out, lse = psa.psa_attn(dq, dk, dv, kbar, vsum, rp_dev, ci_dev, ws=ws, row_max=rmax_t, want_lse=True)
+    status = psa.psa_read_status(ws)
+    g = dict(out=out.cpu(), lse=lse.cpu(), row_ptr=rp_t, col_idx=ci_t, status=status)
+    _, kb, vs = O.pool(f64(q), f64(k), f64(v))
+    check_output(g, q, k, v, kb, vs, False, sample_units(B, H, M, 30, seed=8, g=g))
+
+
+def test_two_streams_match_serial_runs():
+    # two problems on two streams at once (own workspaces and outputs) give
+    # bit-identical results to the same calls made one after the other
+    probs = [make_qkv(1, 3, 48 * 64, 128, "clustered", seed=s) for s in (24, 25)]
+    devs = [tuple(x.cuda() for x in p) for p in probs]
+    B, H, N, d = probs[0][0].shape
+    wss = [psa.workspace(B, H, N, d) for _ in range(2)]
+    serial = []
+    for (q, k, v), ws in zip(devs, wss):
+        out, _ = psa.psa_forward(q, k, v, mode="topk", density=0.2, ws=ws)
+        torch.cuda.synchronize()
+        serial.append(out.clone())
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    outs = []
+    for (q, k, v), ws, s in zip(devs, wss, streams):
+        with torch.cuda.stream(s):
+            out, _ = psa.psa_forward(q, k, v, mode="topk", density=0.2, ws=ws, stream=s)
+        outs.append(out)
+    torch.cuda.synchronize()
+    for a, b, ws in zip(outs, serial, wss):
+        assert psa.psa_read_status(ws) == psa.PSA_OK
+        assert torch.equal(a, b)
