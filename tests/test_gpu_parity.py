@@ -353,3 +353,26 @@ def test_two_streams_match_serial_runs():
     for a, b, ws in zip(outs, serial, wss):
         assert psa.psa_read_status(ws) == psa.PSA_OK
         assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------ dense at full size
+@pytest.mark.parametrize("name", ["dit_video_n32k", "long_causal_n128k"])
+def test_full_size_dense_sampled(name):
+    # psa_dense (every candidate block exact) at a full workload shape, against
+    # the oracle with every candidate listed on a sample of query blocks
+    w = WORKLOADS[name]
+    q, k, v = workload_inputs(name)
+    H = 2  # two heads of the workload keep the host side quick
+    q, k, v = q[:, :H].contiguous(), k[:, :H].contiguous(), v[:, :H].contiguous()
+    B, _, N, d = q.shape
+    M = N // 64
+    causal = w["causal"]
+    dq, dk, dv = (x.cuda() for x in (q, k, v))
+    ws = psa.workspace(B, H, N, d)
+    out, lse = psa.psa_dense(dq, dk, dv, causal, ws=ws, want_lse=True)
+    status = psa.psa_read_status(ws)
+    lists = [np.arange(I + 1 if causal else M) for _ in range(B * H) for I in range(M)]
+    rp, ci = O._to_csr(lists)
+    g = dict(out=out.cpu(), lse=lse.cpu(), row_ptr=rp, col_idx=ci, status=status)
+    _, kb, vs = O.pool(f64(q), f64(k), f64(v))
+    check_output(g, q, k, v, kb, vs, causal, sample_units(B, H, M, 16, seed=9))
