@@ -32,8 +32,10 @@
 //    Warp group 0: warp 0 loads Q and K tiles, warp 2 loads V tiles (TMA);
 //    warp 1 issues S^T = K.Q^T and owns TMEM, warp 3 issues O^T += V^T.P^T
 //    (one thread each).  Warp groups 1 and 2 take alternate tiles for the
-//    softmax, one thread per TMEM lane (= key row of S^T), and share the
-//    epilogue (one thread per feature row of O^T).  Two S^T buffers and two
+//    softmax, one thread per TMEM lane (= key row of S^T); at a unit's end
+//    the one that does not own the next unit's first tile writes the output
+//    alone (one thread per feature row of O^T) while the other starts that
+//    tile.  Two S^T buffers and two
 //    O^T accumulators (by unit parity) let consecutive tiles and units
 //    overlap.
 //  * Every wait is bounded; on a timeout all roles stop, drain what is in
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = bars + 12;   // P^T written                   (4 warps)
   uint64_t* g2_done = bars + 14;  // GEMM2 done: V stage and P^T buffer free (commit)
   uint64_t* o_full = bars + 16;   // last GEMM2 of the unit done   (commit)
-  uint64_t* o_empty = bars + 18;  // O^T read by the epilogue      (8 warps)
+  uint64_t* o_empty = bars + 18;  // O^T read by the epilogue      (4 warps)
   uint64_t* drain = bars + 20;    // [2] teardown of the two issuers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[i], 4);
       mbar_init(&g2_done[i], 1);
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], 8);
+      mbar_init(&o_empty[i], 4);   // the warps of one softmax warpgroup
       mbar_init(&drain[i], 1);
     }
     *abort_flag = 0;
@@ -683,10 +685,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + gtid] = (c2 + __log2f(l)) * kLn2;
       }
       const bool more = u + static_cast<int>(gridDim.x) < p.units;
-      if (gtid == 0) {
-        bulk_wait_read0();  // the previous unit's store has read the staging tile
-        *stop_s = *abort_flag;
-      }
+      if (gtid == 0) *stop_s = *abort_flag;
+      if ((gtid & 127) == 0) bulk_wait_read0();  // the last unit's store has read the staging tile
       if (more && !p.dense)
         for (int i = gtid; i < nw_all; i += 256) bitmap[i] = 0u;
       named_barrier_sync(1, 256);
@@ -697,34 +697,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         load_next(u + gridDim.x);
         prologue(u + gridDim.x, na, nb, nrmax);
       }
-      const int ob = ul & 1;
-      mbar_wait(&o_full[ob], (ul >> 1) & 1, abort_flag, p.status);
-      tc_fence_after();
-      if (trow < D) {  // warp-uniform; warpgroup w stores queries [32 w, 32 w + 32)
-        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sOut);
-        float ov[32];
-        tmem_ld32(tbase + lane_addr + 128 + 64 * ob + 32 * w, ov);
-        tc_wait_ld();
+      // the output: the warpgroup that does not own the next unit's first
+      // tile writes all 64 query columns while the other goes on
+      if (w != (sc & 1)) {
+        const int ob = ul & 1;
+        mbar_wait(&o_full[ob], (ul >> 1) & 1, abort_flag, p.status);
+        tc_fence_after();
+        if (trow < D) {  // warp-uniform
+          __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sOut);
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            float ov[32];
+            tmem_ld32(tbase + lane_addr + 128 + 64 * ob + 32 * h, ov);
+            tc_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          st[(32 * w + q) * D + trow] = __float2bfloat16_rn(ov[q] * invl[32 * w + q]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[ob]);
-      fence_async_shared();
-      named_barrier_sync(1, 256);
-      if (gtid == 0) {
-        bulk_store(p.out + static_cast<size_t>(row_done) * 64 * D, sOut, C::kOutBytes);
-        bulk_commit();
-        if (*unit_flag) {
-          const int slot = atomicAdd(p.fixup_count, 1);
-          p.fixup_list[slot] = u;
-          *unit_flag = 0;
+            for (int q = 0; q < 32; ++q)
+              st[(32 * h + q) * D + trow] = __float2bfloat16_rn(ov[q] * invl[32 * h + q]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_empty[ob]);
+        fence_async_shared();
+        named_barrier_sync(2 + w, 128);
+        if ((gtid & 127) == 0) {
+          bulk_store(p.out + static_cast<size_t>(row_done) * 64 * D, sOut, C::kOutBytes);
+          bulk_commit();
+          if (*unit_flag) {
+            const int slot = atomicAdd(p.fixup_count, 1);
+            p.fixup_list[slot] = u;
+            *unit_flag = 0;
+          }
         }
       }
     }
-    if (gtid == 0) bulk_wait0();
+    if ((gtid & 127) == 0) bulk_wait0();
   }
 
   tc_fence_before();
