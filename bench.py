@@ -181,8 +181,15 @@ class Step:
         self.out = torch.empty_like(self.q)
         self.out_host = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
         self.stream = torch.cuda.current_stream()
-        # kernels of ours launched by one step
-        self.launches = 3 if dense else 1 + (1 if self.mode == "topk" else 3) + 3
+        # kernels of ours launched by one step: pool; route = two operand splits,
+        # then per batch of heads one score and one selection launch (the library
+        # batches as many heads as fit 256 MB of scores), + scan and compaction
+        # for the threshold routers; attention = 3
+        Mp = -(-self.M // 128) * 128
+        per_batch = max(1, min(B * H, (256 << 20) // (self.M * Mp * 4)))
+        nb = -(-(B * H) // per_batch)
+        route = 2 + 2 * nb + (0 if self.mode == "topk" else 2)
+        self.launches = 3 if dense else 1 + route + 3
 
     def run(self, ev=None, io=None, stream=None):
         """pool -> route -> attention; ``ev`` = 4 events to split the kernels;
@@ -207,7 +214,7 @@ class Step:
             ev[1].record(s)
         qbar, kbar, vsum = self.stats
         if self.mode == "topk":
-            psa.psa_route_topk(qbar, kbar, self.param, self.causal, out=self.csr, stream=s)
+            psa.psa_route_topk(qbar, kbar, self.param, self.causal, out=self.csr, ws=self.ws, stream=s)
         elif self.mode == "thresh_prob":
             psa.psa_route_thresh_prob(qbar, kbar, self.param, self.causal, self.keep_first, ws=self.ws,
                                       out=self.csr, stream=s)

@@ -27,6 +27,16 @@ WorkspaceLayout workspace_layout(long long BH, long long M, long long d) {
   o += align256(static_cast<size_t>(BH * M) * 4);
   L.row_bits = o;
   o += align256(static_cast<size_t>(BH * M * ((M + 31) / 32)) * 4);
+  L.q_split = o;
+  o += align256(static_cast<size_t>(3 * BH * M * d) * 2);
+  L.k_split = o;
+  o += align256(static_cast<size_t>(3 * BH * M * d) * 2);
+  // block scores of as many heads as fit 256 MB (at least one)
+  const size_t head_scores = static_cast<size_t>(M) * score_stride(static_cast<int>(M)) * 4;
+  const long long fit = static_cast<long long>((size_t(256) << 20) / head_scores);
+  L.score_heads = static_cast<int>(fit < 1 ? 1 : (fit > BH ? BH : fit));
+  L.scores = o;
+  o += align256(head_scores * L.score_heads);
   L.total = o;
   return L;
 }
@@ -110,6 +120,16 @@ long long causal_prefix(long long I, long long k0) {
 
 namespace {
 
+psa::RouteScratch route_scratch(char* ws, const psa::WorkspaceLayout& L) {
+  psa::RouteScratch w;
+  w.q_split = reinterpret_cast<uint16_t*>(ws + L.q_split);
+  w.k_split = reinterpret_cast<uint16_t*>(ws + L.k_split);
+  w.scores = reinterpret_cast<float*>(ws + L.scores);
+  w.heads_per_batch = L.score_heads;
+  w.status = reinterpret_cast<int*>(ws + L.header);
+  return w;
+}
+
 // Shared by both threshold routers: thr_I = a_mul * max_J s_IJ + a_add.
 int route_thresh_common(const float* qbar, const float* kbar, int B, int H, int M, int d, float a_mul, float a_add,
                         int causal, int keep_first, int* row_ptr, int* col_idx, size_t capacity, int* nnz_out,
@@ -128,11 +148,13 @@ int route_thresh_common(const float* qbar, const float* kbar, int B, int H, int 
   if ((s = check_device()) != PSA_OK) return s;
   const long long cap = capacity > static_cast<size_t>(INT_MAX) ? INT_MAX : static_cast<long long>(capacity);
   char* ws = static_cast<char*>(workspace);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
   return cuda_status(psa::launch_route_thresh(qbar, kbar, static_cast<int>(bh), M, d, a_mul, a_add, causal,
                                               keep_first, row_ptr, col_idx, cap, nnz_out,
                                               reinterpret_cast<int*>(ws + L.row_count),
                                               reinterpret_cast<uint32_t*>(ws + L.row_bits), row_max,
-                                              static_cast<cudaStream_t>(stream)));
+                                              route_scratch(ws, L), st));
 }
 
 }  // namespace
@@ -154,7 +176,7 @@ const char* psa_status_string(int status) {
   }
 }
 
-int psa_version(void) { return 100; }
+int psa_version(void) { return 200; }
 
 size_t psa_workspace_size(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d, kBlock) != PSA_OK) return 0;
@@ -181,8 +203,9 @@ int psa_pool(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int 
 }
 
 int psa_route_topk(const float* qbar, const float* kbar, int B, int H, int M, int d, float density, int causal,
-                   int* row_ptr, int* col_idx, size_t capacity, int* nnz_out, float* row_max, void* stream) {
-  if (!qbar || !kbar || !row_ptr || !col_idx || !nnz_out) return PSA_ERR_ARG;
+                   int* row_ptr, int* col_idx, size_t capacity, int* nnz_out, float* row_max, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (!qbar || !kbar || !row_ptr || !col_idx || !nnz_out || !workspace) return PSA_ERR_ARG;
   if (reinterpret_cast<uintptr_t>(row_max) & 3u) return PSA_ERR_ARG;
   if (M <= 0) return PSA_ERR_ARG;
   if (M > kMaxBlocks) return PSA_ERR_UNSUPPORTED;
@@ -190,7 +213,7 @@ int psa_route_topk(const float* qbar, const float* kbar, int B, int H, int M, in
   if (s != PSA_OK) return s;
   if (!(density >= 0.0f) || std::isinf(density)) return PSA_ERR_ARG;
   if (causal != 0 && causal != 1) return PSA_ERR_ARG;
-  if (!aligned16(qbar) || !aligned16(kbar)) return PSA_ERR_ARG;
+  if (!aligned16(qbar) || !aligned16(kbar) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PSA_ERR_ARG;
   // k = clamp(ceil(fl32(density * M)), 1, #candidates): single-precision product
   volatile float prod = density * static_cast<float>(M);
   double kc = std::ceil(static_cast<double>(prod));
@@ -198,10 +221,15 @@ int psa_route_topk(const float* qbar, const float* kbar, int B, int H, int M, in
   const long long bh = static_cast<long long>(B) * H;
   const long long total = causal ? bh * causal_prefix(M, k0) : bh * M * k0;
   if (total > INT_MAX || static_cast<size_t>(total) > capacity) return PSA_ERR_CAPACITY;
+  const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
+  if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
   if ((s = check_device()) != PSA_OK) return s;
+  char* ws = static_cast<char*>(workspace);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
   return cuda_status(psa::launch_route_topk(qbar, kbar, static_cast<int>(bh), M, d, static_cast<int>(k0),
                                             causal, row_ptr, col_idx, total, nnz_out, row_max,
-                                            static_cast<cudaStream_t>(stream)));
+                                            route_scratch(ws, L), st));
 }
 
 int psa_route_thresh(const float* qbar, const float* kbar, int B, int H, int M, int d, float alpha, int causal,

@@ -21,9 +21,33 @@ struct WorkspaceLayout {
   size_t vsum_bf16 = 0;     // bf16 [B*H*M*d] (value sums)
   size_t row_count = 0;     // int [B*H*M]     (threshold routing)
   size_t row_bits = 0;      // uint32 [B*H*M*ceil(M/32)]
+  size_t q_split = 0;       // bf16 [3][B*H*M*d] (three-part split of qbar, routing)
+  size_t k_split = 0;       // bf16 [3][B*H*M*d] (same for kbar)
+  size_t scores = 0;        // fp32 [score_heads][M][Mp] block scores of one batch of heads
+  int score_heads = 0;      // heads per routing batch
   size_t total = 0;
 };
 WorkspaceLayout workspace_layout(long long BH, long long M, long long d);
+
+// Routing scratch inside the workspace.
+struct RouteScratch {
+  uint16_t* q_split;
+  uint16_t* k_split;
+  float* scores;
+  int heads_per_batch;
+  int* status;
+};
+
+// score.cu: block scores s_IJ = qbar_I . kbar_J / sqrt(d) on the tensor cores
+int score_stride(int M);  // Mp: M rounded up to the 128-column score tile
+cudaError_t launch_split3(const float* x, long long n, uint16_t* out, cudaStream_t st);
+struct ScorePlan {
+  CUtensorMap mq, mk;  // the split operands, 128-row x 64-feature boxes
+  int BH = 0, M = 0, d = 0, Mp = 0;
+  cudaError_t init(const uint16_t* q_split, const uint16_t* k_split, int BH, int M, int d);
+  // scores of heads [bh0, bh0 + nh) into scores[nh][M][Mp]
+  cudaError_t run(int bh0, int nh, int causal, float* scores, int* status, cudaStream_t st) const;
+};
 
 // pool.cu
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int M, int d,
@@ -36,12 +60,12 @@ cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long
 // route.cu
 cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int M, int d, int k0, int causal,
                               int* row_ptr, int* col_idx, long long total, int* nnz_out, float* row_max,
-                              cudaStream_t st);
+                              const RouteScratch& w, cudaStream_t st);
 // threshold thr_I = a_mul * max_J s_IJ + a_add (one fma)
 cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, int M, int d, float a_mul,
                                 float a_add, int causal, int keep_first, int* row_ptr, int* col_idx, long long capacity,
                                 int* nnz_out, int* row_count, uint32_t* row_bits, float* row_max,
-                                cudaStream_t st);
+                                const RouteScratch& w, cudaStream_t st);
 
 // attn.cu
 struct AttnLaunch {

@@ -1,20 +1,21 @@
-// route.cu -- a2..a4: block scores and the two routers.
+// route.cu -- a3/a4: the two routers, on the block scores of score.cu.
 //
 // Scores: PISA summary (kodorricoding.tistory.com/108), "How are candidate
 // blocks narrowed": one score per (query block, key block) from the block
-// representatives, s_IJ = qbar_I . kbar_J / sqrt(d), computed in fp32.
-// Top-k: the same section and the usage line (`density`).  Threshold:
-// FlashPrefill summary, 2.b "Max-based dynamic thresholding",
-// thresh_I = alpha * max_J s_IJ, no sort and no cumulative sum.
+// representatives, s_IJ = qbar_I . kbar_J / sqrt(d), computed at fp32
+// accuracy on the tensor cores (score.cu).  Top-k: the same section and the
+// usage line (`density`).  Threshold: FlashPrefill summary, 2.b "Max-based
+// dynamic thresholding", thresh_I = alpha * max_J s_IJ, no sort and no
+// cumulative sum.
 //
-// A CTA of 256 threads scores R consecutive query blocks of one head against
-// every candidate key block (kbar rows are read once per CTA and reused for
-// the R rows), keeps the scores in shared memory, and then one warp per row
-// selects.  Top-k finds the k-th largest score exactly by a 32-step bitwise
-// search over the order-preserving integer image of the fp32 scores (ties
-// resolved by ascending J), so it needs no sort; both routers write the
-// list in ascending J with warp ballots, and, when asked, each row's largest
-// candidate score (the attention step's softmax stabiliser).
+// A CTA of 256 threads copies the score rows of R consecutive query blocks
+// of one head into shared memory, and then one warp per row selects.  Top-k
+// finds the k-th largest score exactly by a 32-step bitwise search over the
+// order-preserving integer image of the fp32 scores (ties resolved by
+// ascending J), so it needs no sort; both routers write the list in
+// ascending J with warp ballots, and, when asked, each row's largest
+// candidate score (the attention step's softmax stabiliser).  Heads are
+// routed in batches whose score matrices fit the workspace.
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -39,104 +40,39 @@ __host__ __device__ inline long long causal_prefix(long long I, long long k0) {
   return k0 * (k0 + 1) / 2 + (I - k0) * k0;
 }
 
-// Scores of rows [I0, I0 + rows) of head bh into ss[r * M + J], J < jmax.
-// Thread t owns key J0 + t of each 256-key chunk and accumulates its R dot
-// products over the features in order.  The kbar rows reach it through
-// shared memory, 16 features of 256 keys at a time: loaded with coalesced
-// 16-byte loads (read straight from global memory, every lane of a warp
-// would touch a different cache line) into rows padded to 20 floats, so the
-// per-thread 16-byte reads are free of bank conflicts.  The next slice is
-// fetched into registers while the current one is consumed.
-constexpr int kSliceF = 16;            // features per slice
-constexpr int kSliceStride = 20;       // padded row, floats
-constexpr int kChunkJ = 256;           // keys per chunk (one per thread)
-
-template <int R, int D>
-__device__ void score_rows(const float* __restrict__ qbar, const float* __restrict__ kbar, int bh, int M,
-                           int I0, int rows, int jmax, float tau, float* sq, float* sk, float* ss) {
-  static_assert(D % kSliceF == 0, "slices");
-  constexpr int kSlices = D / kSliceF;
-  const int tid = threadIdx.x;
-  for (int e = tid; e < R * D; e += blockDim.x)
-    sq[e] = e < rows * D ? qbar[(static_cast<size_t>(bh) * M + I0) * D + e] : 0.f;
-  const float* kb = kbar + static_cast<size_t>(bh) * M * D;
-  const float4* sq4 = reinterpret_cast<const float4*>(sq);
-  for (int J0 = 0; J0 < jmax; J0 += kChunkJ) {
-    // slice loader: float4 e = i * 256 + tid covers key row e / 4, features 4 (e % 4) ..
-    float4 pre[4];
-    auto fetch = [&](int s) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int e = i * 256 + tid, row = e >> 2, c4 = e & 3;
-        pre[i] = J0 + row < jmax
-                     ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(J0 + row) * D + s * kSliceF) + c4)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    };
-    auto stash = [&](float* buf) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int e = i * 256 + tid, row = e >> 2, c4 = e & 3;
-        *reinterpret_cast<float4*>(buf + row * kSliceStride + 4 * c4) = pre[i];
-      }
-    };
-    float acc[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = 0.f;
-    fetch(0);
-    __syncthreads();  // previous chunk's readers are done with both buffers
-    stash(sk);
-#pragma unroll 1
-    for (int s = 0; s < kSlices; ++s) {
-      float* cur = sk + (s & 1) * kChunkJ * kSliceStride;
-      if (s + 1 < kSlices) fetch(s + 1);
-      __syncthreads();
-      const float4* kr = reinterpret_cast<const float4*>(cur + tid * kSliceStride);
-#pragma unroll
-      for (int c = 0; c < kSliceF / 4; ++c) {
-        const float4 kv = kr[c];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const float4 qv = sq4[r * (D / 4) + s * (kSliceF / 4) + c];
-          acc[r] = fmaf(qv.x, kv.x, acc[r]);
-          acc[r] = fmaf(qv.y, kv.y, acc[r]);
-          acc[r] = fmaf(qv.z, kv.z, acc[r]);
-          acc[r] = fmaf(qv.w, kv.w, acc[r]);
-        }
-      }
-      if (s + 1 < kSlices) stash(sk + ((s + 1) & 1) * kChunkJ * kSliceStride);
-    }
-    const int J = J0 + tid;
-    if (J < jmax) {
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-        if (r < rows) ss[r * M + J] = acc[r] * tau + 0.0f;  // +0 folds -0 into +0
-    }
+// Score rows [I0, I0 + rows) of local head hl, candidates J < jmax, into
+// ss[r * Mp + J] (row stride Mp, a multiple of 128, so the copy moves float4s).
+template <int R>
+__device__ void load_rows(const float* __restrict__ scores, int M, int Mp, int hl, int I0, int rows, int jmax,
+                          float* ss) {
+  const int q4 = (jmax + 3) / 4, per = Mp / 4;
+  const float4* src = reinterpret_cast<const float4*>(scores + (static_cast<size_t>(hl) * M + I0) * Mp);
+  float4* dst = reinterpret_cast<float4*>(ss);
+  for (int e = threadIdx.x; e < rows * per; e += blockDim.x) {
+    const int r = e / per, c = e - r * per;
+    if (c < q4) dst[e] = __ldg(src + static_cast<size_t>(r) * per + c);
   }
   __syncthreads();
 }
 
-template <int R, int D>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ qbar,
-                                                         const float* __restrict__ kbar, int BH, int M,
-                                                         float tau, int k0, int causal, int* __restrict__ row_ptr,
-                                                         int* __restrict__ col_idx, long long total,
-                                                         int* __restrict__ nnz_out, float* __restrict__ row_max) {
-  extern __shared__ float sm[];
-  const int bh = blockIdx.y;
+template <int R>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ scores, int Mp, int bh0,
+                                                         int BH, int M, int k0, int causal,
+                                                         int* __restrict__ row_ptr, int* __restrict__ col_idx,
+                                                         long long total, int* __restrict__ nnz_out,
+                                                         float* __restrict__ row_max) {
+  extern __shared__ float ss[];
+  const int hl = blockIdx.y, bh = bh0 + hl;
   const int I0 = blockIdx.x * R;
   const int rows = min(R, M - I0);
   const int jmax = causal ? min(M, I0 + rows) : M;
-  float* sq = sm;
-  float* sk = sq + R * D;
-  float* ss = sk + 2 * kChunkJ * kSliceStride;
-  score_rows<R, D>(qbar, kbar, bh, M, I0, rows, jmax, tau, sq, sk, ss);
+  load_rows<R>(scores, M, Mp, hl, I0, rows, jmax, ss);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (warp >= rows) return;
   const int I = I0 + warp;
   const long long row = static_cast<long long>(bh) * M + I;
-  const float* s = ss + warp * M;
+  const float* s = ss + warp * Mp;
   const int cand = causal ? I + 1 : M;
   const int kk = max(1, min(k0, cand));
   // causal: the diagonal takes one slot, the rest come from J < I
@@ -204,29 +140,25 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   }
 }
 
-template <int R, int D>
-__global__ void __launch_bounds__(256) route_thresh_kernel(const float* __restrict__ qbar,
-                                                           const float* __restrict__ kbar, int M,
-                                                           float tau, float a_mul, float a_add, int causal,
+template <int R>
+__global__ void __launch_bounds__(256) route_thresh_kernel(const float* __restrict__ scores, int Mp, int bh0,
+                                                           int M, float a_mul, float a_add, int causal,
                                                            int keep_first,
                                                            int* __restrict__ row_count,
                                                            uint32_t* __restrict__ row_bits,
                                                            float* __restrict__ row_max) {
-  extern __shared__ float sm[];
-  const int bh = blockIdx.y;
+  extern __shared__ float ss[];
+  const int hl = blockIdx.y, bh = bh0 + hl;
   const int I0 = blockIdx.x * R;
   const int rows = min(R, M - I0);
   const int jmax = causal ? min(M, I0 + rows) : M;
-  float* sq = sm;
-  float* sk = sq + R * D;
-  float* ss = sk + 2 * kChunkJ * kSliceStride;
-  score_rows<R, D>(qbar, kbar, bh, M, I0, rows, jmax, tau, sq, sk, ss);
+  load_rows<R>(scores, M, Mp, hl, I0, rows, jmax, ss);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (warp >= rows) return;
   const int I = I0 + warp;
   const long long row = static_cast<long long>(bh) * M + I;
-  const float* s = ss + warp * M;
+  const float* s = ss + warp * Mp;
   const int cand = causal ? I + 1 : M;
   float m = -INFINITY;
   for (int J = lane; J < cand; J += 32) m = fmaxf(m, s[J]);
@@ -332,14 +264,12 @@ __global__ void __launch_bounds__(256) compact_rows_kernel(const uint32_t* __res
   }
 }
 
-// shared memory of a router CTA: R query rows, the two kbar slices, R score rows
-size_t route_smem(int R, int M, int d) {
-  return (static_cast<size_t>(R) * (M + d) + 2 * kChunkJ * kSliceStride) * sizeof(float);
-}
+// shared memory of a router CTA: R score rows of stride Mp
+size_t route_smem(int R, int Mp) { return static_cast<size_t>(R) * Mp * sizeof(float); }
 
-int rows_per_cta(int M, int d) {
+int rows_per_cta(int Mp) {
   for (int R = 8; R > 1; R >>= 1)
-    if (route_smem(R, M, d) <= 200 * 1024) return R;
+    if (route_smem(R, Mp) <= 200 * 1024) return R;
   return 1;
 }
 
@@ -348,73 +278,83 @@ cudaError_t set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
+// Split both operands and prepare the score tiles of every head.
+cudaError_t prepare_scores(const float* qbar, const float* kbar, int BH, int M, int d, const RouteScratch& w,
+                           ScorePlan& plan, cudaStream_t st) {
+  if (d != 64 && d != 128) return cudaErrorInvalidValue;
+  const long long n = static_cast<long long>(BH) * M * d;
+  cudaError_t e;
+  if ((e = launch_split3(qbar, n, w.q_split, st)) != cudaSuccess) return e;
+  if ((e = launch_split3(kbar, n, w.k_split, st)) != cudaSuccess) return e;
+  return plan.init(w.q_split, w.k_split, BH, M, d);
+}
+
 }  // namespace
 
 cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int M, int d, int k0, int causal,
                               int* row_ptr, int* col_idx, long long total, int* nnz_out, float* row_max,
-                              cudaStream_t st) {
-  const int R = rows_per_cta(M, d);
-  const size_t smem = route_smem(R, M, d);
-  const dim3 grid((M + R - 1) / R, BH);
-  const float tau = 1.0f / sqrtf(static_cast<float>(d));
-  cudaError_t e;
-#define PSA_TOPK(RR)                                                                                   \
-  case RR:                                                                                             \
-    if (d == 128) {                                                                                    \
-      if ((e = set_smem(route_topk_kernel<RR, 128>, smem)) != cudaSuccess) return e;                   \
-      route_topk_kernel<RR, 128><<<grid, 256, smem, st>>>(qbar, kbar, BH, M, tau, k0, causal, row_ptr, \
-                                                           col_idx, total, nnz_out, row_max);          \
-    } else {                                                                                           \
-      if ((e = set_smem(route_topk_kernel<RR, 64>, smem)) != cudaSuccess) return e;                    \
-      route_topk_kernel<RR, 64><<<grid, 256, smem, st>>>(qbar, kbar, BH, M, tau, k0, causal, row_ptr,  \
-                                                          col_idx, total, nnz_out, row_max);           \
-    }                                                                                                  \
+                              const RouteScratch& w, cudaStream_t st) {
+  ScorePlan plan;
+  cudaError_t e = prepare_scores(qbar, kbar, BH, M, d, w, plan, st);
+  if (e != cudaSuccess) return e;
+  const int Mp = plan.Mp;
+  const int R = rows_per_cta(Mp);
+  const size_t smem = route_smem(R, Mp);
+  for (int h0 = 0; h0 < BH; h0 += w.heads_per_batch) {
+    const int nh = BH - h0 < w.heads_per_batch ? BH - h0 : w.heads_per_batch;
+    if ((e = plan.run(h0, nh, causal, w.scores, w.status, st)) != cudaSuccess) return e;
+    const dim3 grid((M + R - 1) / R, nh);
+#define PSA_TOPK(RR)                                                                                         \
+  case RR:                                                                                                   \
+    if ((e = set_smem(route_topk_kernel<RR>, smem)) != cudaSuccess) return e;                                \
+    route_topk_kernel<RR><<<grid, 256, smem, st>>>(w.scores, Mp, h0, BH, M, k0, causal, row_ptr, col_idx,    \
+                                                   total, nnz_out, row_max);                                 \
     break;
-  if (d != 64 && d != 128) return cudaErrorInvalidValue;
-  switch (R) {
-    PSA_TOPK(8)
-    PSA_TOPK(4)
-    PSA_TOPK(2)
-    PSA_TOPK(1)
-    default:
-      return cudaErrorInvalidValue;
-  }
+    switch (R) {
+      PSA_TOPK(8)
+      PSA_TOPK(4)
+      PSA_TOPK(2)
+      PSA_TOPK(1)
+      default:
+        return cudaErrorInvalidValue;
+    }
 #undef PSA_TOPK
-  return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, int M, int d, float a_mul,
                                 float a_add, int causal, int keep_first, int* row_ptr, int* col_idx, long long capacity,
                                 int* nnz_out, int* row_count, uint32_t* row_bits, float* row_max,
-                                cudaStream_t st) {
-  const int R = rows_per_cta(M, d);
-  const size_t smem = route_smem(R, M, d);
-  const dim3 grid((M + R - 1) / R, BH);
-  const float tau = 1.0f / sqrtf(static_cast<float>(d));
-  cudaError_t e;
-#define PSA_THRESH(RR)                                                                                 \
-  case RR:                                                                                             \
-    if (d == 128) {                                                                                    \
-      if ((e = set_smem(route_thresh_kernel<RR, 128>, smem)) != cudaSuccess) return e;                 \
-      route_thresh_kernel<RR, 128><<<grid, 256, smem, st>>>(qbar, kbar, M, tau, a_mul, a_add, causal,  \
-                                                             keep_first, row_count, row_bits, row_max); \
-    } else {                                                                                           \
-      if ((e = set_smem(route_thresh_kernel<RR, 64>, smem)) != cudaSuccess) return e;                  \
-      route_thresh_kernel<RR, 64><<<grid, 256, smem, st>>>(qbar, kbar, M, tau, a_mul, a_add, causal,   \
-                                                            keep_first, row_count, row_bits, row_max);  \
-    }                                                                                                  \
+                                const RouteScratch& w, cudaStream_t st) {
+  ScorePlan plan;
+  cudaError_t e = prepare_scores(qbar, kbar, BH, M, d, w, plan, st);
+  if (e != cudaSuccess) return e;
+  const int Mp = plan.Mp;
+  const int R = rows_per_cta(Mp);
+  const size_t smem = route_smem(R, Mp);
+  for (int h0 = 0; h0 < BH; h0 += w.heads_per_batch) {
+    const int nh = BH - h0 < w.heads_per_batch ? BH - h0 : w.heads_per_batch;
+    if ((e = plan.run(h0, nh, causal, w.scores, w.status, st)) != cudaSuccess) return e;
+    const dim3 grid((M + R - 1) / R, nh);
+#define PSA_THRESH(RR)                                                                                       \
+  case RR:                                                                                                   \
+    if ((e = set_smem(route_thresh_kernel<RR>, smem)) != cudaSuccess) return e;                              \
+    route_thresh_kernel<RR><<<grid, 256, smem, st>>>(w.scores, Mp, h0, M, a_mul, a_add, causal, keep_first,  \
+                                                     row_count, row_bits, row_max);                          \
     break;
-  if (d != 64 && d != 128) return cudaErrorInvalidValue;
-  switch (R) {
-    PSA_THRESH(8)
-    PSA_THRESH(4)
-    PSA_THRESH(2)
-    PSA_THRESH(1)
-    default:
-      return cudaErrorInvalidValue;
-  }
+    switch (R) {
+      PSA_THRESH(8)
+      PSA_THRESH(4)
+      PSA_THRESH(2)
+      PSA_THRESH(1)
+      default:
+        return cudaErrorInvalidValue;
+    }
 #undef PSA_THRESH
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   const long long nrows = static_cast<long long>(BH) * M;
   scan_rows_kernel<<<1, 1024, 0, st>>>(row_count, nrows, capacity, row_ptr, nnz_out);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -49,7 +49,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "psa_workspace_size": (Z, [I, I, I, I]),
         "psa_route_capacity": (Z, [I, I, I, I]),
         "psa_pool": (I, [P, P, P, I, I, I, I, I, P, P, P, P]),
-        "psa_route_topk": (I, [P, P, I, I, I, I, F, I, P, P, Z, P, P, P]),
+        "psa_route_topk": (I, [P, P, I, I, I, I, F, I, P, P, Z, P, P, P, Z, P]),
         "psa_route_thresh": (I, [P, P, I, I, I, I, F, I, I, P, P, Z, P, P, P, Z, P]),
         "psa_route_thresh_prob": (I, [P, P, I, I, I, I, F, I, I, P, P, Z, P, P, P, Z, P]),
         "psa_attn": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, Z, P]),
@@ -144,17 +144,19 @@ def _route_out(B, H, M, causal, capacity, device):
 
 
 def psa_route_topk(qbar, kbar, density: float, causal: bool = False, capacity: int | None = None,
-                   out=None, stream=None):
+                   out=None, ws=None, stream=None):
     """Returns (row_ptr, col_idx, nnz, row_max): device int32 tensors (nnz has
     one element) and the float32 row maxima of the block scores (``out`` may
     give row_max as None to skip it)."""
     B, H, M, d = (int(x) for x in qbar.shape)
+    if ws is None:
+        ws = workspace(B, H, M * 64, d, qbar.device)
     if out is None:
         out = _route_out(B, H, M, causal, capacity, qbar.device)
     row_ptr, col_idx, nnz, row_max = out
     _check("psa_route_topk", lib().psa_route_topk(
         _ptr(qbar), _ptr(kbar), B, H, M, d, float(density), int(causal), _ptr(row_ptr), _ptr(col_idx),
-        col_idx.numel(), _ptr(nnz), _ptr(row_max), _stream(stream)))
+        col_idx.numel(), _ptr(nnz), _ptr(row_max), _ptr(ws), ws.numel(), _stream(stream)))
     return row_ptr, col_idx, nnz, row_max
 
 
@@ -264,7 +266,7 @@ def psa_forward(q, k, v, mode: str = "topk", density: float = 0.15, alpha: float
         ws = workspace(B, H, N, d, q.device)
     qbar, kbar, vsum = psa_pool(q, k, v, stream=stream)
     if mode == "topk":
-        csr = psa_route_topk(qbar, kbar, density, causal, stream=stream)
+        csr = psa_route_topk(qbar, kbar, density, causal, ws=ws, stream=stream)
     elif mode == "thresh":
         csr = psa_route_thresh(qbar, kbar, alpha, causal, keep_first, ws=ws, stream=stream)
     elif mode == "thresh_prob":

@@ -64,8 +64,10 @@ PSA_API const char* psa_status_string(int status);
 PSA_API int psa_version(void);
 
 /*
- * Bytes of device workspace that psa_route_thresh, psa_attn and psa_dense
- * need for a problem of this shape (one workspace serves all three).  The
+ * Bytes of device workspace that the routers, psa_attn and psa_dense need
+ * for a problem of this shape (one workspace serves them all).  Besides
+ * O(B*H*M*d) of pooled data it holds the block-score matrices of as many
+ * heads as fit 256 MB (at least one head: 4*M*ceil(M/128)*128 bytes).  The
  * workspace must be 256-byte aligned and is owned by the caller; calls that
  * share one workspace must be ordered on one stream.  Returns 0 for invalid
  * sizes.
@@ -104,13 +106,21 @@ PSA_API int psa_pool(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
  * *nnz_out (device int32) = total listed, and, when row_max is not NULL,
  * row_max [B*H*M] (device float32) = max over the candidates of s_IJ, the
  * softmax stabiliser psa_attn can take instead of computing its own.
+ * `workspace` (device, 256-byte aligned, psa_workspace_size(B,H,64*M,d)
+ * bytes) holds the score matrices: the scores are one tensor-core product
+ * per head at fp32 accuracy (each fp32 operand split into three bf16 parts),
+ * written to the workspace and then selected from; heads go in batches that
+ * fit it.  The call resets the workspace status word; a bounded device wait
+ * that runs out records PSA_ERR_TIMEOUT there (psa_read_status).
  * Errors: PSA_ERR_ARG, PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY (capacity
- * below the exact total, which the host knows for top-k), PSA_ERR_CUDA.
+ * below the exact total, which the host knows for top-k, or workspace too
+ * small), PSA_ERR_CUDA.
  */
 PSA_API int psa_route_topk(const float* qbar, const float* kbar,
                    int B, int H, int M, int d, float density, int causal,
                    int* row_ptr, int* col_idx, size_t capacity, int* nnz_out,
-                   float* row_max, void* stream);
+                   float* row_max, void* workspace, size_t workspace_bytes,
+                   void* stream);
 
 /*
  * a2 + a4. Block scores and sorting-free threshold routing [FlashPrefill
@@ -122,9 +132,11 @@ PSA_API int psa_route_topk(const float* qbar, const float* kbar,
  * (row_ptr stays a valid, truncated CSR) and the caller must retry with a
  * larger col_idx.  psa_route_capacity() never overflows.  row_max
  * (nullable) as for psa_route_topk: the row maxima the threshold is taken of.
- * `workspace` (device, psa_workspace_size(B,H,64*M,d) bytes) holds the row
- * counts and bit masks between the three launches.  Errors: PSA_ERR_ARG,
- * PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY (workspace too small), PSA_ERR_CUDA.
+ * `workspace` (device, psa_workspace_size(B,H,64*M,d) bytes) holds the
+ * score matrices (as for psa_route_topk) and the row counts and bit masks
+ * between the launches; the call resets its status word.  Errors:
+ * PSA_ERR_ARG, PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY (workspace too small),
+ * PSA_ERR_CUDA.
  */
 PSA_API int psa_route_thresh(const float* qbar, const float* kbar,
                      int B, int H, int M, int d, float alpha, int causal,
@@ -232,8 +244,8 @@ PSA_API int psa_test_stall_next_attn(int on);
 /*
  * Synchronises `stream`, then copies the device status word of `workspace`
  * into *status (host pointer): PSA_OK, or the first device-side error
- * recorded since the last call that reset it (psa_route_thresh, psa_attn
- * and psa_dense reset it at their start).  Returns PSA_OK or PSA_ERR_CUDA.
+ * recorded since the last call that reset it (the routers, psa_attn and
+ * psa_dense reset it at their start).  Returns PSA_OK or PSA_ERR_CUDA.
  */
 PSA_API int psa_read_status(const void* workspace, int* status, void* stream);
 

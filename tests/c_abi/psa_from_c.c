@@ -74,7 +74,8 @@ int main(int argc, char** argv) {
   CHECK_CUDA(cudaMemcpyAsync(q, host, 3 * n * sizeof(psa_bf16_t), cudaMemcpyHostToDevice, stream));
 
   CHECK_PSA(psa_pool(q, k, v, B, H, N, d, 64, qbar, kbar, vsum, stream));
-  CHECK_PSA(psa_route_topk(qbar, kbar, B, H, M, d, density, 0, row_ptr, col_idx, cap, nnz, row_max, stream));
+  CHECK_PSA(psa_route_topk(qbar, kbar, B, H, M, d, density, 0, row_ptr, col_idx, cap, nnz, row_max, ws,
+                           ws_bytes, stream));
   CHECK_PSA(psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, cap, row_max, B, H, N, d, 64, 0, out, NULL, ws,
                      ws_bytes, stream));
   int device_status = -1;

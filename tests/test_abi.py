@@ -64,12 +64,21 @@ def test_host_validation_rejects_bad_arguments():
     assert L.psa_pool(ctypes.c_void_p((1 << 20) + 2), FAKE, FAKE, 1, 1, 64, 64, 64, FAKE, FAKE, FAKE, S) \
         == psa.PSA_ERR_ARG
     # top-k: capacity below the exact total, bad density
-    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 2 * 16 * 4 - 1, FAKE, None, S) \
-        == psa.PSA_ERR_CAPACITY
-    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, float("nan"), 0, FAKE, FAKE, 1 << 20, FAKE, None, S) \
+    big = 1 << 40
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 2 * 16 * 4 - 1, FAKE, None, FAKE, big,
+                            S) == psa.PSA_ERR_CAPACITY
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, float("nan"), 0, FAKE, FAKE, 1 << 20, FAKE, None, FAKE, big,
+                            S) == psa.PSA_ERR_ARG
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 2, FAKE, FAKE, 1 << 20, FAKE, None, FAKE, big, S) \
         == psa.PSA_ERR_ARG
-    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 2, FAKE, FAKE, 1 << 20, FAKE, None, S) \
+    # top-k: workspace missing, misaligned, too small
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 1 << 20, FAKE, None, None, big, S) \
         == psa.PSA_ERR_ARG
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 1 << 20, FAKE, None,
+                            ctypes.c_void_p((1 << 20) + 16), big, S) == psa.PSA_ERR_ARG
+    need = psa.psa_workspace_size(1, 2, 16 * 64, 64)
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 1 << 20, FAKE, None, FAKE, need - 1,
+                            S) == psa.PSA_ERR_CAPACITY
     # threshold: workspace too small, bad alpha
     assert L.psa_route_thresh(FAKE, FAKE, 1, 2, 16, 64, 0.5, 0, 0, FAKE, FAKE, 1 << 20, FAKE, None, FAKE, 16, S) \
         == psa.PSA_ERR_CAPACITY
@@ -91,7 +100,7 @@ def test_host_validation_rejects_bad_arguments():
                                    S) == psa.PSA_ERR_CAPACITY
     # misaligned row maxima (routers' output, attention's input)
     odd = ctypes.c_void_p((1 << 20) + 2)
-    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 1 << 20, FAKE, odd, S) \
+    assert L.psa_route_topk(FAKE, FAKE, 1, 2, 16, 64, 0.25, 0, FAKE, FAKE, 1 << 20, FAKE, odd, FAKE, 1 << 40, S) \
         == psa.PSA_ERR_ARG
     assert L.psa_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, odd, 1, 2, 1024, 64, 64, 0, FAKE,
                       None, FAKE, ws, S) == psa.PSA_ERR_ARG
