@@ -40,7 +40,9 @@ struct RouteScratch {
 
 // score.cu: block scores s_IJ = qbar_I . kbar_J / sqrt(d) on the tensor cores
 int score_stride(int M);  // Mp: M rounded up to the 128-column score tile
-cudaError_t launch_split3(const float* x, long long n, uint16_t* out, cudaStream_t st);
+// three-way bf16 split of two fp32 arrays of n values each, in one launch
+cudaError_t launch_split3(const float* x0, const float* x1, long long n, uint16_t* out0, uint16_t* out1,
+                          cudaStream_t st);
 struct ScorePlan {
   CUtensorMap mq, mk;  // the split operands, 128-row x 64-feature boxes
   int BH = 0, M = 0, d = 0, Mp = 0;

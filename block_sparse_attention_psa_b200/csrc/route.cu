@@ -33,6 +33,54 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Inverse of order_key.
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// One histogram step of the radix select: lanes with the same digit add
+// once (digit 256 = this lane has no key in play).
+__device__ __forceinline__ void hist_add(int* hist, int lane, int digit) {
+  const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+  if (digit < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+}
+
+// The bucket of a 256-bucket histogram that holds the need-th largest key
+// (counting from the top bucket down): its digit, and how many keys the
+// buckets above it hold.  Lane l scans buckets 255 - 8l down to 248 - 8l.
+__device__ __forceinline__ void pick_bucket(const int* hist, int lane, int need, int& digit, int& above) {
+  int c[8], sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = hist[255 - 8 * lane - i];
+    sum += c[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int excl = incl - sum;
+  const bool mine = excl < need && incl >= need;
+  const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+  int dg = 0, ab = 0;
+  if (mine) {
+    int run = excl;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (run + c[i] >= need) {
+        dg = 255 - 8 * lane - i;
+        ab = run;
+        break;
+      }
+      run += c[i];
+    }
+  }
+  digit = __shfl_sync(0xffffffffu, dg, src);
+  above = __shfl_sync(0xffffffffu, ab, src);
+}
+
 // Sum over i < I of min(k0, i + 1): start of row I inside its head for causal
 // top-k (k0 >= 1).
 __host__ __device__ inline long long causal_prefix(long long I, long long k0) {
@@ -40,70 +88,99 @@ __host__ __device__ inline long long causal_prefix(long long I, long long k0) {
   return k0 * (k0 + 1) / 2 + (I - k0) * k0;
 }
 
-// Score rows [I0, I0 + rows) of local head hl, candidates J < jmax, into
-// ss[r * Mp + J] (row stride Mp, a multiple of 128, so the copy moves float4s).
-template <int R>
-__device__ void load_rows(const float* __restrict__ scores, int M, int Mp, int hl, int I0, int rows, int jmax,
-                          float* ss) {
-  const int q4 = (jmax + 3) / 4, per = Mp / 4;
-  const float4* src = reinterpret_cast<const float4*>(scores + (static_cast<size_t>(hl) * M + I0) * Mp);
-  float4* dst = reinterpret_cast<float4*>(ss);
-  for (int e = threadIdx.x; e < rows * per; e += blockDim.x) {
-    const int r = e / per, c = e - r * per;
-    if (c < q4) dst[e] = __ldg(src + static_cast<size_t>(r) * per + c);
+// Score row I0 + warp of local head hl, candidates J < jmax, into
+// ss[warp * Mp + J]: each warp copies the row it then selects from (row
+// stride Mp, a multiple of 128, so the copy moves coalesced float4s).  With
+// Keys the row is stored as the order keys of the scores.
+template <bool Keys>
+__device__ __forceinline__ void load_row(const float* __restrict__ scores, int M, int Mp, int hl, int I, int jmax,
+                                         float* ss_row) {
+  const int lane = threadIdx.x % 32;
+  const int q4 = (jmax + 3) / 4;
+  const float4* src = reinterpret_cast<const float4*>(scores + (static_cast<size_t>(hl) * M + I) * Mp);
+  float4* dst = reinterpret_cast<float4*>(ss_row);
+  auto put = [&](int c, float4 x) {
+    if (Keys)
+      x = make_float4(__uint_as_float(order_key(x.x)), __uint_as_float(order_key(x.y)),
+                      __uint_as_float(order_key(x.z)), __uint_as_float(order_key(x.w)));
+    dst[c] = x;
+  };
+  int c = lane;
+  for (; c + 96 < q4; c += 128) {
+    const float4 x0 = __ldg(src + c), x1 = __ldg(src + c + 32), x2 = __ldg(src + c + 64), x3 = __ldg(src + c + 96);
+    put(c, x0);
+    put(c + 32, x1);
+    put(c + 64, x2);
+    put(c + 96, x3);
   }
-  __syncthreads();
+  for (; c < q4; c += 32) put(c, __ldg(src + c));
+  __syncwarp();
 }
 
 template <int R>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ scores, int Mp, int bh0,
+__global__ void __launch_bounds__(256, 4) route_topk_kernel(const float* __restrict__ scores, int Mp, int bh0,
                                                          int BH, int M, int k0, int causal,
                                                          int* __restrict__ row_ptr, int* __restrict__ col_idx,
                                                          long long total, int* __restrict__ nnz_out,
                                                          float* __restrict__ row_max) {
-  extern __shared__ float ss[];
+  extern __shared__ float ss[];  // [R][Mp] score rows, then [R][256] histograms
   const int hl = blockIdx.y, bh = bh0 + hl;
   const int I0 = blockIdx.x * R;
   const int rows = min(R, M - I0);
-  const int jmax = causal ? min(M, I0 + rows) : M;
-  load_rows<R>(scores, M, Mp, hl, I0, rows, jmax, ss);
-
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (warp >= rows) return;
   const int I = I0 + warp;
-  const long long row = static_cast<long long>(bh) * M + I;
-  const float* s = ss + warp * Mp;
   const int cand = causal ? I + 1 : M;
+  load_row<true>(scores, M, Mp, hl, I, cand, ss + warp * Mp);
+  const long long row = static_cast<long long>(bh) * M + I;
+  const uint32_t* sk = reinterpret_cast<const uint32_t*>(ss + warp * Mp);  // order keys
+  int* hist = reinterpret_cast<int*>(ss + R * Mp) + warp * 256;
   const int kk = max(1, min(k0, cand));
   // causal: the diagonal takes one slot, the rest come from J < I
   const int n = causal ? I : M;
   const int krest = causal ? kk - 1 : kk;
   if (row_max) {
-    float m = -INFINITY;
-    for (int J = lane; J < cand; J += 32) m = fmaxf(m, s[J]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) row_max[row] = m;
+    uint32_t mk = 0;
+    for (int J = lane; J < cand; J += 32) mk = max(mk, sk[J]);
+    mk = __reduce_max_sync(0xffffffffu, mk);
+    if (lane == 0) row_max[row] = key_float(mk);
   }
 
+  // T = the krest-th largest order key among J < n, exactly: a radix
+  // select over four 8-bit digits, high to low.  Each pass histograms the
+  // digit of the keys that share the prefix fixed so far (lanes holding
+  // the same digit add once, through a match), then finds the bucket that
+  // holds the krest-th key by a scan from the top bucket down.
   uint32_t T = 0;
   if (krest > 0) {
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t t = T | (1u << bit);
-      int cnt = 0;
-      for (int J = lane; J < n; J += 32) cnt += order_key(s[J]) >= t;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= krest) {
-        T = t;
-        // exactly krest keys are >= T: they are the selection (every key equal
-        // to T is in it, so the tie rule below takes them all)
-        if (cnt == krest) break;
+    uint32_t prefix = 0;
+    int need = krest;  // rank of T among the keys that share `prefix`
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int b = lane; b < 256; b += 32) hist[b] = 0;
+      __syncwarp();
+      const uint32_t hi = shift == 24 ? 0u : 0xffffffffu << (shift + 8);
+      for (int J0 = 0; J0 < n; J0 += 32) {
+        const int J = J0 + lane;
+        int digit = 256;  // no key
+        if (J < n) {
+          const uint32_t key = sk[J];
+          if ((key & hi) == prefix) digit = static_cast<int>((key >> shift) & 255u);
+        }
+        hist_add(hist, lane, digit);
       }
+      __syncwarp();
+      int digit, above;
+      pick_bucket(hist, lane, need, digit, above);
+      prefix |= static_cast<uint32_t>(digit) << shift;
+      need -= above;
+      __syncwarp();
     }
+    T = prefix;
   }
   int gt = 0;
   if (krest > 0)
-    for (int J = lane; J < n; J += 32) gt += order_key(s[J]) > T;
+    for (int J = lane; J < n; J += 32) gt += sk[J] > T;
   gt = __reduce_add_sync(0xffffffffu, gt);
   const int need_eq = krest - gt;
 
@@ -120,7 +197,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     const int J = J0 + lane;
     bool gtf = false, eqf = false;
     if (J < n && krest > 0) {
-      const uint32_t key = order_key(s[J]);
+      const uint32_t key = sk[J];
       gtf = key > T;
       eqf = key == T;
     }
@@ -141,25 +218,23 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 }
 
 template <int R>
-__global__ void __launch_bounds__(256) route_thresh_kernel(const float* __restrict__ scores, int Mp, int bh0,
+__global__ void __launch_bounds__(256, 4) route_thresh_kernel(const float* __restrict__ scores, int Mp, int bh0,
                                                            int M, float a_mul, float a_add, int causal,
                                                            int keep_first,
                                                            int* __restrict__ row_count,
                                                            uint32_t* __restrict__ row_bits,
                                                            float* __restrict__ row_max) {
-  extern __shared__ float ss[];
+  extern __shared__ float ss[];  // [R][Mp] score rows
   const int hl = blockIdx.y, bh = bh0 + hl;
   const int I0 = blockIdx.x * R;
   const int rows = min(R, M - I0);
-  const int jmax = causal ? min(M, I0 + rows) : M;
-  load_rows<R>(scores, M, Mp, hl, I0, rows, jmax, ss);
-
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (warp >= rows) return;
   const int I = I0 + warp;
+  const int cand = causal ? I + 1 : M;
+  load_row<false>(scores, M, Mp, hl, I, cand, ss + warp * Mp);
   const long long row = static_cast<long long>(bh) * M + I;
   const float* s = ss + warp * Mp;
-  const int cand = causal ? I + 1 : M;
   float m = -INFINITY;
   for (int J = lane; J < cand; J += 32) m = fmaxf(m, s[J]);
 #pragma unroll
@@ -264,8 +339,9 @@ __global__ void __launch_bounds__(256) compact_rows_kernel(const uint32_t* __res
   }
 }
 
-// shared memory of a router CTA: R score rows of stride Mp
-size_t route_smem(int R, int Mp) { return static_cast<size_t>(R) * Mp * sizeof(float); }
+// shared memory of a router CTA: R score rows of stride Mp (+ R 256-bucket
+// histograms for top-k)
+size_t route_smem(int R, int Mp) { return static_cast<size_t>(R) * (Mp + 256) * sizeof(float); }
 
 int rows_per_cta(int Mp) {
   for (int R = 8; R > 1; R >>= 1)
@@ -283,9 +359,8 @@ cudaError_t prepare_scores(const float* qbar, const float* kbar, int BH, int M, 
                            ScorePlan& plan, cudaStream_t st) {
   if (d != 64 && d != 128) return cudaErrorInvalidValue;
   const long long n = static_cast<long long>(BH) * M * d;
-  cudaError_t e;
-  if ((e = launch_split3(qbar, n, w.q_split, st)) != cudaSuccess) return e;
-  if ((e = launch_split3(kbar, n, w.k_split, st)) != cudaSuccess) return e;
+  const cudaError_t e = launch_split3(qbar, kbar, n, w.q_split, w.k_split, st);
+  if (e != cudaSuccess) return e;
   return plan.init(w.q_split, w.k_split, BH, M, d);
 }
 

@@ -297,6 +297,18 @@ def test_maximum_block_count():
         psa.PSA_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("M,causal", [(1024, False), (1024, True), (1100, False), (1100, True)])
+def test_topk_selection_on_both_sides_of_1024_candidates(M, causal):
+    # rows of up to 1024 candidates are selected with their keys in registers,
+    # longer rows from shared memory: both against the oracle on every row
+    q, k, v = make_qkv(1, 2, M * 64, 64, "clustered", seed=23)
+    g = run_gpu(q, k, v, "topk", 0.1, causal)
+    assert g["status"] == psa.PSA_OK
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    check_routing(g, O.block_scores(qbar, kbar), "topk", 0.1, causal)
+    check_output(g, q, k, v, kbar, vsum, causal, sample_units(1, 2, M, 8, seed=7, g=g))
+
+
 # ------------------------------------------------------------------ capacity and streams
 def test_threshold_truncation_keeps_a_valid_prefix():
     # a col_idx buffer half the exact total: the exact total is still reported,
