@@ -400,7 +400,9 @@ def gpu_arm(args):
         "roofline": {"bound": "tensor",
                      "kernel": "attn_kernel (psa_dense call)" if st.dense else "attn_kernel (psa_attn call)",
                      "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / tc_peak, 4), "traffic": recorded_traffic(st.name),
+                     "frac": round(achieved / tc_peak, 4),
+                     # the capture is of psa_attn at the workload's own routing
+                     "traffic": None if st.dense or args.density is not None else recorded_traffic(st.name),
                      "peak_source": peaks["source"] + " bf16 burst"},
         "kernels": {"pool_ms": None if st.dense else round(pool_avg, 4),
                     "route_ms": None if st.dense else round(route_avg, 4), "attn_ms": round(attn_avg, 4),
