@@ -181,15 +181,7 @@ class Step:
         self.out = torch.empty_like(self.q)
         self.out_host = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
         self.stream = torch.cuda.current_stream()
-        # kernels of ours launched by one step: pool; route = two operand splits,
-        # then per batch of heads one score and one selection launch (the library
-        # batches as many heads as fit 256 MB of scores), + scan and compaction
-        # for the threshold routers; attention = 3
-        Mp = -(-self.M // 128) * 128
-        per_batch = max(1, min(B * H, (256 << 20) // (self.M * Mp * 4)))
-        nb = -(-(B * H) // per_batch)
-        route = 2 + 2 * nb + (0 if self.mode == "topk" else 2)
-        self.launches = 3 if dense else 1 + route + 3
+        self.launches = launches_per_step(B, H, self.M, self.mode, dense)
 
     def run(self, ev=None, io=None, stream=None):
         """pool -> route -> attention; ``ev`` = 4 events to split the kernels;
@@ -271,6 +263,22 @@ class Step:
 
     def d2h_bytes(self):
         return self.out_host.numel() * self.out_host.element_size()
+
+
+def launches_per_step(B: int, H: int, M: int, mode: str, dense: bool) -> int:
+    """Kernels of ours one step launches: psa_dense = 3 (key pooling,
+    attention, fixup); otherwise pool 1, route = one split of both operands
+    plus, per batch of heads, one score and one selection launch (the library
+    batches as many heads as fit 256 MB of scores), plus scan and compaction
+    for the threshold routers, and attention 3 (bf16 statistics, attention,
+    fixup)."""
+    if dense:
+        return 3
+    Mp = -(-M // 128) * 128
+    per_batch = max(1, min(B * H, (256 << 20) // (M * Mp * 4)))
+    nb = -(-(B * H) // per_batch)
+    route = 1 + 2 * nb + (0 if mode == "topk" else 2)
+    return 1 + route + 3
 
 
 def _flush(buf):

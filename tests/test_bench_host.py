@@ -57,3 +57,14 @@ def test_issued_flops_counts_tiles():
 def test_dense_flops_formula():
     assert bench.dense_flops(2, 3, 128, 64, False) == 4.0 * 2 * 3 * 128 * 128 * 64
     assert bench.dense_flops(2, 3, 128, 64, True) == 2.0 * 2 * 3 * 128 * 128 * 64
+
+
+def test_launches_per_step_matches_the_launch_lists():
+    # launch lists of one step (pool, split3, score_tc, selection, stats_to_bf16,
+    # attention, fixup; + scan and compaction for the threshold routers)
+    assert bench.launches_per_step(1, 12, 512, "topk", False) == 7
+    assert bench.launches_per_step(1, 12, 512, "thresh", False) == 9
+    assert bench.launches_per_step(1, 8, 2048, "thresh", False) == 9      # 8 x 16 MB of scores: one batch
+    assert bench.launches_per_step(1, 1, 16384, "topk", False) == 7
+    assert bench.launches_per_step(1, 2, 16384, "topk", False) == 9       # 1 GB per head: two batches
+    assert bench.launches_per_step(1, 12, 512, "topk", True) == 3
