@@ -139,19 +139,18 @@ __global__ void __launch_bounds__(256, 4) route_topk_kernel(const float* __restr
   // causal: the diagonal takes one slot, the rest come from J < I
   const int n = causal ? I : M;
   const int krest = causal ? kk - 1 : kk;
-  if (row_max) {
-    uint32_t mk = 0;
-    for (int J = lane; J < cand; J += 32) mk = max(mk, sk[J]);
-    mk = __reduce_max_sync(0xffffffffu, mk);
-    if (lane == 0) row_max[row] = key_float(mk);
-  }
-
   // T = the krest-th largest order key among J < n, exactly: a radix
   // select over four 8-bit digits, high to low.  Each pass histograms the
   // digit of the keys that share the prefix fixed so far (lanes holding
   // the same digit add once, through a match), then finds the bucket that
-  // holds the krest-th key by a scan from the top bucket down.
+  // holds the krest-th key by a scan from the top bucket down.  The keys in
+  // the buckets above the chosen ones are exactly the keys above T, so the
+  // rank left at the end is the number of keys equal to T to take.  The
+  // first pass also takes the row maximum (the diagonal J = I = n is the
+  // one candidate outside J < n, when causal).
   uint32_t T = 0;
+  int need_eq = 0;
+  uint32_t mk = causal ? sk[I] : 0u;
   if (krest > 0) {
     uint32_t prefix = 0;
     int need = krest;  // rank of T among the keys that share `prefix`
@@ -165,6 +164,7 @@ __global__ void __launch_bounds__(256, 4) route_topk_kernel(const float* __restr
         int digit = 256;  // no key
         if (J < n) {
           const uint32_t key = sk[J];
+          if (shift == 24) mk = max(mk, key);
           if ((key & hi) == prefix) digit = static_cast<int>((key >> shift) & 255u);
         }
         hist_add(hist, lane, digit);
@@ -177,12 +177,14 @@ __global__ void __launch_bounds__(256, 4) route_topk_kernel(const float* __restr
       __syncwarp();
     }
     T = prefix;
+    need_eq = need;
+  } else if (row_max) {
+    for (int J = lane; J < n; J += 32) mk = max(mk, sk[J]);
   }
-  int gt = 0;
-  if (krest > 0)
-    for (int J = lane; J < n; J += 32) gt += sk[J] > T;
-  gt = __reduce_add_sync(0xffffffffu, gt);
-  const int need_eq = krest - gt;
+  if (row_max) {
+    mk = __reduce_max_sync(0xffffffffu, mk);
+    if (lane == 0) row_max[row] = key_float(mk);
+  }
 
   long long start;
   if (causal) {

@@ -40,7 +40,7 @@ def run_gpu(q, k, v, mode, param, causal=False, keep_first=False, want_lse=True,
     ws = psa.workspace(B, H, N, d)
     qbar, kbar, vsum = psa.psa_pool(dq, dk, dv)
     if mode == "topk":
-        row_ptr, col_idx, nnz, row_max = psa.psa_route_topk(qbar, kbar, param, causal)
+        row_ptr, col_idx, nnz, row_max = psa.psa_route_topk(qbar, kbar, param, causal, ws=ws)
     elif mode == "thresh_prob":
         row_ptr, col_idx, nnz, row_max = psa.psa_route_thresh_prob(qbar, kbar, param, causal, keep_first, ws=ws)
     else:

@@ -309,6 +309,19 @@ def test_topk_selection_on_both_sides_of_1024_candidates(M, causal):
     check_output(g, q, k, v, kbar, vsum, causal, sample_units(1, 2, M, 8, seed=7, g=g))
 
 
+@pytest.mark.parametrize("mode,param", [("topk", 0.004), ("thresh", 0.5)])
+def test_routing_in_two_head_batches(mode, param):
+    # M = 8192: one head's scores fill the 256 MB the workspace holds, so the
+    # two heads are scored and selected in two batches (second at head offset 1)
+    M, d = 8192, 64
+    q, k, v = make_qkv(1, 2, M * 64, d, "clustered", seed=24)
+    g = run_gpu(q, k, v, mode, param)
+    assert g["status"] == psa.PSA_OK
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    check_routing(g, O.block_scores(qbar, kbar), mode, param, False)
+    check_output(g, q, k, v, kbar, vsum, False, sample_units(1, 2, M, 8, seed=8, g=g))
+
+
 # ------------------------------------------------------------------ capacity and streams
 def test_threshold_truncation_keeps_a_valid_prefix():
     # a col_idx buffer half the exact total: the exact total is still reported,
