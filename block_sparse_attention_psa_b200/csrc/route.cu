@@ -141,9 +141,8 @@ __global__ void __launch_bounds__(256, 4) route_topk_kernel(const float* __restr
   const int krest = causal ? kk - 1 : kk;
   // T = the krest-th largest order key among J < n, exactly: a radix
   // select over four 8-bit digits, high to low.  Each pass histograms the
-  // digit of the keys that share the prefix fixed so far (lanes holding
-  // the same digit add once, through a match), then finds the bucket that
-  // holds the krest-th key by a scan from the top bucket down.  The keys in
+  // digit of the keys that share the prefix fixed so far, then finds the
+  // bucket that holds the krest-th key by a scan from the top bucket down.  The keys in
   // the buckets above the chosen ones are exactly the keys above T, so the
   // rank left at the end is the number of keys equal to T to take.  The
   // first pass also takes the row maximum (the diagonal J = I = n is the
@@ -159,15 +158,25 @@ __global__ void __launch_bounds__(256, 4) route_topk_kernel(const float* __restr
       for (int b = lane; b < 256; b += 32) hist[b] = 0;
       __syncwarp();
       const uint32_t hi = shift == 24 ? 0u : 0xffffffffu << (shift + 8);
-      for (int J0 = 0; J0 < n; J0 += 32) {
-        const int J = J0 + lane;
-        int digit = 256;  // no key
-        if (J < n) {
-          const uint32_t key = sk[J];
-          if (shift == 24) mk = max(mk, key);
-          if ((key & hi) == prefix) digit = static_cast<int>((key >> shift) & 255u);
+      if (shift == 24) {
+        // first digit (sign and leading exponent bits): keys crowd into a
+        // few values, so lanes with equal digits add once
+        for (int J0 = 0; J0 < n; J0 += 32) {
+          const int J = J0 + lane;
+          int digit = 256;  // no key
+          if (J < n) {
+            const uint32_t key = sk[J];
+            mk = max(mk, key);
+            digit = static_cast<int>(key >> 24);
+          }
+          hist_add(hist, lane, digit);
         }
-        hist_add(hist, lane, digit);
+      } else {
+        // later digits: only keys with the prefix count, and they rarely collide
+        for (int J = lane; J < n; J += 32) {
+          const uint32_t key = sk[J];
+          if ((key & hi) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        }
       }
       __syncwarp();
       int digit, above;
