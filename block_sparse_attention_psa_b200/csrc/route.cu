@@ -38,13 +38,6 @@ __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// One histogram step of the radix select: lanes with the same digit add
-// once (digit 256 = this lane has no key in play).
-__device__ __forceinline__ void hist_add(int* hist, int lane, int digit) {
-  const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-  if (digit < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
-}
-
 // The bucket of a 256-bucket histogram that holds the need-th largest key
 // (counting from the top bucket down): its digit, and how many keys the
 // buckets above it hold.  Lane l scans buckets 255 - 8l down to 248 - 8l.
@@ -159,8 +152,7 @@ __global__ void __launch_bounds__(256, 4) route_topk_kernel(const float* __restr
       __syncwarp();
       const uint32_t hi = shift == 24 ? 0u : 0xffffffffu << (shift + 8);
       if (shift == 24) {
-        // first digit (sign and leading exponent bits): keys crowd into a
-        // few values, so lanes with equal digits add once
+        // first digit (sign and leading exponent bits): every key counts
         for (int J0 = 0; J0 < n; J0 += 32) {
           const int J = J0 + lane;
           int digit = 256;  // no key
@@ -169,10 +161,10 @@ __global__ void __launch_bounds__(256, 4) route_topk_kernel(const float* __restr
             mk = max(mk, key);
             digit = static_cast<int>(key >> 24);
           }
-          hist_add(hist, lane, digit);
+          if (digit < 256) atomicAdd(&hist[digit], 1);
         }
       } else {
-        // later digits: only keys with the prefix count, and they rarely collide
+        // later digits: only the keys that share the prefix count
         for (int J = lane; J < n; J += 32) {
           const uint32_t key = sk[J];
           if ((key & hi) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
