@@ -61,6 +61,15 @@ Readings where the pages are silent (each is listed in the design doc):
   exp(a_iJ) * (b for the denominator, sum_j v_j for the numerator), with
   a_iJ = q_i . k-bar_J / sqrt(d).
 
+* first-order term (``attention_first_order``, oracle only so far): the
+  expansion of e^{q.k_j/sqrt(d)} to first order around the block-mean key;
+  the pages' "global statistic H" is read as the mean over the head's blocks
+  of the per-block matrices H_J = sum_j (k_j - kbar_J) v_j^T;
+* FlashPrefill's fused "score then pool" block score (the token queries of
+  block I against the pooled key of block J, reduced over I in one pass,
+  ``token_pooled_block_scores``) is read with mean pooling, which makes it
+  equal to qbar_I . kbar_J / sqrt(d) by linearity.
+
 Parity of the approximate output to the authors' own implementation is
 unpinned (no page prints a worked PISA example); the oracle is pinned to the
 definitions above by the tests in ``tests/test_oracle_pins.py``.
@@ -79,9 +88,14 @@ __all__ = [
     "topk_count",
     "route_topk",
     "route_thresh",
+    "route_thresh_prob",
     "attention",
     "attention_online",
     "unit_rows",
+    "block_deviation_stats",
+    "global_deviation_stat",
+    "attention_first_order",
+    "token_pooled_block_scores",
 ]
 
 
@@ -361,3 +375,104 @@ def attention_online(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool,
         out[n] = o / l[:, None]
         lse[n] = m + np.log(l)
     return out, lse
+
+
+# --------------------------------------------------------------------------
+# f-1. First-order term of the unselected blocks
+#   [PISA summary, "Why approximating unselected blocks keeps softmax intact":
+#    to the 0th-order term around the block-mean key a first-order
+#    correction with a global statistic H is added; FAQ "Why a global
+#    first-order correction?": one global statistic instead of re-reading a
+#    large matrix per block]
+# --------------------------------------------------------------------------
+def block_deviation_stats(k, v, block_size: int = 64):
+    """H_J = sum_{j in J} (k_j - kbar_J) v_j^T for every block J.
+
+    Returns ``[B, H, M, d, d]`` float64 (rows: key features, columns: value
+    features)."""
+    k, v = _f64(k), _f64(v)
+    B, H, N, d = k.shape
+    if N % block_size:
+        raise ValueError("N must be a multiple of block_size")
+    M = N // block_size
+    kb = k.reshape(B, H, M, block_size, d)
+    vb = v.reshape(B, H, M, block_size, d)
+    dev = kb - kb.mean(axis=3, keepdims=True)
+    return np.einsum("bhmtk,bhmtv->bhmkv", dev, vb)
+
+
+def global_deviation_stat(HJ):
+    """The global statistic, read as the mean of H_J over a head's blocks:
+    ``[B, H, d, d]``."""
+    return _f64(HJ).mean(axis=2)
+
+
+def _first_order_numerator(ea, Qi, Hs, d):
+    """sum_J e^{a_iJ - m_i} (H_J^T q_i) / sqrt(d) for the query rows ``Qi``
+    [b, d], the weights ``ea`` [b, n_unsel] and the statistics ``Hs``
+    [n_unsel, d, d] of the unselected blocks."""
+    return np.einsum("iJ,ik,Jkv->iv", ea, Qi, Hs) / math.sqrt(d)
+
+
+def attention_first_order(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool, Hstat,
+                          block_size: int = 64, units=None):
+    """The 0th-order output of :func:`attention` with the first-order term of
+    every unselected block added.
+
+    To first order around the block-mean key,
+      e^{q.k_j/sqrt(d)} ~= e^{a_J} (1 + q.(k_j - kbar_J)/sqrt(d)),
+    and the deviations k_j - kbar_J sum to zero over the block, so the
+    denominator term stays block_size * e^{a_J} while the numerator term
+    becomes e^{a_J} (vsum_J + H_J^T q / sqrt(d)).  ``Hstat`` is either the
+    per-block ``[B, H, M, d, d]`` of :func:`block_deviation_stats` (the
+    expansion itself) or one ``[B, H, d, d]`` matrix per head used for every
+    block (the global statistic).  Same max and shapes as :func:`attention`.
+    """
+    q, k, v, kbar, vsum, Hstat = map(_f64, (q, k, v, kbar, vsum, Hstat))
+    B, H, N, d = q.shape
+    bs = block_size
+    M = N // bs
+    per_block = Hstat.ndim == 5
+    if units is None:
+        units = unit_rows(B, H, M)
+    units = list(units)
+    out = np.empty((len(units), bs, d))
+    lse = np.empty((len(units), bs))
+    for n, (b, h, I) in enumerate(units):
+        r = (b * H + h) * M + I
+        sel = col_idx[row_ptr[r]:row_ptr[r + 1]]
+        z, Vx, a, VS = _unit_terms(q, k, v, kbar, vsum, sel, b, h, I, causal, bs)
+        n_pseudo = I if causal else candidate_count(I, M, causal)
+        unsel = np.setdiff1d(np.arange(n_pseudo), np.asarray(sel, dtype=np.int64))
+        m = np.full(bs, -np.inf)
+        if z.shape[1]:
+            m = np.maximum(m, z.max(axis=1))
+        if a.shape[1]:
+            m = np.maximum(m, a.max(axis=1))
+        ez = np.exp(z - m[:, None])
+        ea = np.exp(a - m[:, None])
+        Qi = q[b, h, I * bs:(I + 1) * bs]
+        Hs = Hstat[b, h, unsel] if per_block else np.broadcast_to(Hstat[b, h], (unsel.size, d, d))
+        num = ez @ Vx + ea @ VS + _first_order_numerator(ea, Qi, Hs, d)
+        den = ez.sum(axis=1) + bs * ea.sum(axis=1)
+        out[n] = num / den[:, None]
+        lse[n] = m + np.log(den)
+    return out, lse
+
+
+# --------------------------------------------------------------------------
+# FlashPrefill's fused scoring, read with mean pooling
+#   [FlashPrefill summary, 2.a "Block approximation": average-pooled keys as
+#    block representatives; a fused 2D-reduction kernel replaces an explicit
+#    compute-then-pool pass]
+# --------------------------------------------------------------------------
+def token_pooled_block_scores(q, kbar, block_size: int = 64):
+    """score[b, h, I, J] = mean over the tokens i of query block I of
+    q_i . kbar_J / sqrt(d): the token-level scores against the pooled keys,
+    pooled over the query block."""
+    q, kbar = _f64(q), _f64(kbar)
+    B, H, N, d = q.shape
+    M = N // block_size
+    tok = np.matmul(q, np.swapaxes(kbar, -1, -2)) / math.sqrt(d)   # [B, H, N, M]
+    return tok.reshape(B, H, M, block_size, kbar.shape[2]).mean(axis=3)
+
