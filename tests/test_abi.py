@@ -125,3 +125,35 @@ def test_no_cpu_fallback_in_product_package():
                 assert "oracle" not in re.sub(r"#.*|//.*", "", src).replace("oracle.", "ORACLE") or \
                     "import oracle" not in src, fn
                 assert "import oracle" not in src and "from oracle" not in src, fn
+
+
+def test_binding_signatures_match_the_header():
+    """Every PSA_API prototype in include/psa.h against the ctypes signature
+    the binding declares: same arity, and each parameter of the same kind
+    (pointer, int, size_t, float)."""
+    import re
+
+    L = psa.lib()
+    text = open(os.path.join(ROOT, "include", "psa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = re.findall(r"PSA_API\s+([\w\s\*]+?)\s*\b(psa_\w+)\s*\(([^;]*?)\)\s*;", text, flags=re.S)
+    assert {name for _, name, _ in protos} == set(psa.EXPORTS)
+
+    def kind(c_decl):
+        c_decl = " ".join(c_decl.split())
+        if "*" in c_decl:
+            return "ptr"
+        base = c_decl.replace("const ", "").split(" ")[0]
+        return {"int": "int", "size_t": "size_t", "float": "float"}[base]
+
+    ctype_kind = {ctypes.c_void_p: "ptr", ctypes.c_int: "int", ctypes.c_size_t: "size_t",
+                  ctypes.c_float: "float"}
+    for ret, name, params in protos:
+        params = " ".join(params.split())
+        c_params = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+        fn = getattr(L, name)
+        assert len(fn.argtypes) == len(c_params), name
+        for c_decl, t in zip(c_params, fn.argtypes):
+            want = kind(c_decl)
+            got = "ptr" if t not in ctype_kind else ctype_kind[t]   # POINTER(...) types are pointers
+            assert got == want, (name, c_decl, t)
