@@ -35,7 +35,7 @@ Sources (web pages; cited by title and section):
   m <- max(m, max z), l <- l e^{m_old-m} + sum e^{z-m},
   o <- o e^{m_old-m} + sum e^{z-m} v, answer o / l).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * layout ``[B, H, N, d]``; block I = tokens [I*b, (I+1)*b); ``N % b == 0``;
 * q-bar and k-bar are means, the value statistic is the plain sum;
