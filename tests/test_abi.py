@@ -157,3 +157,28 @@ def test_binding_signatures_match_the_header():
             want = kind(c_decl)
             got = "ptr" if t not in ctype_kind else ctype_kind[t]   # POINTER(...) types are pointers
             assert got == want, (name, c_decl, t)
+
+
+def test_workspace_size_holds_the_documented_parts():
+    """psa_workspace_size = pooled data O(B*H*M*d) + threshold masks + the
+    block-score matrices of as many heads as fit 256 MB (at least one head,
+    4*M*Mp bytes, Mp = M rounded up to 128)."""
+    def parts(B, H, M, d):
+        bh = B * H
+        Mp = -(-M // 128) * 128
+        head = 4 * M * Mp
+        heads = max(1, min(bh, (256 << 20) // head))
+        pooled = bh * M * 4 + 2 * bh * M * d * 2 + bh * M * 4 + 2 * 3 * bh * M * d * 2
+        masks = bh * M * (-(-M // 32)) * 4
+        return pooled + masks + heads * head
+
+    for B, H, M, d in ((1, 12, 512, 128), (1, 8, 2048, 128), (1, 24, 1024, 64), (1, 2, 8192, 64),
+                       (1, 1, 16384, 64), (2, 3, 37, 64)):
+        got = psa.psa_workspace_size(B, H, M * 64, d)
+        want = parts(B, H, M, d)
+        # each region is rounded up to 256 bytes (header + 8 regions)
+        assert want <= got <= want + 256 * 10, (B, H, M, d, got, want)
+    # two heads of M = 8192 do not fit 256 MB together: one head's matrix is held
+    one = psa.psa_workspace_size(1, 1, 8192 * 64, 64)
+    two = psa.psa_workspace_size(1, 2, 8192 * 64, 64)
+    assert two - one < 4 * 8192 * 8192
