@@ -68,3 +68,26 @@ def test_launches_per_step_matches_the_launch_lists():
     assert bench.launches_per_step(1, 1, 16384, "topk", False) == 7
     assert bench.launches_per_step(1, 2, 16384, "topk", False) == 9       # 1 GB per head: two batches
     assert bench.launches_per_step(1, 12, 512, "topk", True) == 3
+
+
+def test_reference_arm_prints_its_line_on_the_host():
+    """bench.py --impl reference: the fp64 oracle on the host cores, one JSON
+    line with the fields the reference arm must carry (no GPU needed)."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3",
+                        "--workload", "tiny_iid_n1k"], cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
+    assert d["higher_is_better"] is True and d["config"]["workload"] == "tiny_iid_n1k"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["e2e"]["value"] == d["value"]
