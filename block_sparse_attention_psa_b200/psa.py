@@ -107,6 +107,42 @@ def _shape(q):
     return tuple(int(x) for x in q.shape)
 
 
+def _expect(name, t, like=None, shape=None, dtype=None, min_numel=None):
+    """The C ABI takes plain pointers sized from the problem's dimensions, so
+    every tensor is checked against them here, before any pointer is passed:
+    a smaller or differently typed buffer would be read or written past its
+    end on the device."""
+    if t is None:
+        return
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} needs at least {min_numel} elements, has {t.numel()}")
+    if like is not None and t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, the problem on {like.device}")
+
+
+def _expect_qkv(q, k, v):
+    B, H, N, d = _shape(q)
+    _expect("k", k, q, (B, H, N, d), torch.bfloat16)
+    _expect("v", v, q, (B, H, N, d), torch.bfloat16)
+    return B, H, N, d
+
+
+def _expect_ws(ws, q, B, H, N, d):
+    _expect("ws", ws, q, dtype=torch.uint8, min_numel=psa_workspace_size(B, H, N, d))
+
+
+def _expect_route_out(out, q, BH, M):
+    row_ptr, col_idx, nnz, row_max = out
+    _expect("row_ptr", row_ptr, q, dtype=torch.int32, min_numel=BH * M + 1)
+    _expect("col_idx", col_idx, q, dtype=torch.int32, min_numel=1)
+    _expect("nnz", nnz, q, dtype=torch.int32, min_numel=1)
+    _expect("row_max", row_max, q, dtype=torch.float32, min_numel=BH * M)
+
+
 def psa_workspace_size(B: int, H: int, N: int, d: int) -> int:
     return int(lib().psa_workspace_size(B, H, N, d))
 
@@ -125,14 +161,23 @@ def workspace(B: int, H: int, N: int, d: int, device=None) -> torch.Tensor:
 
 def psa_pool(q, k, v, block_size: int = 64, out=None, stream=None):
     """Returns (qbar, kbar, vsum) float32 [B, H, M, d]."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _expect_qkv(q, k, v)
     M = N // block_size if block_size > 0 else 0
     if out is None:
         out = tuple(torch.empty(B, H, M, d, dtype=torch.float32, device=q.device) for _ in range(3))
     qbar, kbar, vsum = out
+    for name, t in (("qbar", qbar), ("kbar", kbar), ("vsum", vsum)):
+        _expect(name, t, q, (B, H, M, d), torch.float32)
     _check("psa_pool", lib().psa_pool(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, block_size,
                                       _ptr(qbar), _ptr(kbar), _ptr(vsum), _stream(stream)))
     return qbar, kbar, vsum
+
+
+def _expect_stats(qbar, kbar):
+    if qbar.dim() != 4 or qbar.dtype != torch.float32:
+        raise ValueError("qbar, kbar must be float32 [B, H, M, d]")
+    _expect("kbar", kbar, qbar, tuple(qbar.shape), torch.float32)
+    return tuple(int(x) for x in qbar.shape)
 
 
 def _route_out(B, H, M, causal, capacity, device):
@@ -148,11 +193,13 @@ def psa_route_topk(qbar, kbar, density: float, causal: bool = False, capacity: i
     """Returns (row_ptr, col_idx, nnz, row_max): device int32 tensors (nnz has
     one element) and the float32 row maxima of the block scores (``out`` may
     give row_max as None to skip it)."""
-    B, H, M, d = (int(x) for x in qbar.shape)
+    B, H, M, d = _expect_stats(qbar, kbar)
     if ws is None:
         ws = workspace(B, H, M * 64, d, qbar.device)
     if out is None:
         out = _route_out(B, H, M, causal, capacity, qbar.device)
+    _expect_ws(ws, qbar, B, H, M * 64, d)
+    _expect_route_out(out, qbar, B * H, M)
     row_ptr, col_idx, nnz, row_max = out
     _check("psa_route_topk", lib().psa_route_topk(
         _ptr(qbar), _ptr(kbar), B, H, M, d, float(density), int(causal), _ptr(row_ptr), _ptr(col_idx),
@@ -163,11 +210,13 @@ def psa_route_topk(qbar, kbar, density: float, causal: bool = False, capacity: i
 def psa_route_thresh(qbar, kbar, alpha: float, causal: bool = False, keep_first: bool = False,
                      ws=None, capacity: int | None = None, out=None, stream=None):
     """Returns (row_ptr, col_idx, nnz, row_max); nnz > col_idx.numel() means truncated."""
-    B, H, M, d = (int(x) for x in qbar.shape)
+    B, H, M, d = _expect_stats(qbar, kbar)
     if ws is None:
         ws = workspace(B, H, M * 64, d, qbar.device)
     if out is None:
         out = _route_out(B, H, M, causal, capacity, qbar.device)
+    _expect_ws(ws, qbar, B, H, M * 64, d)
+    _expect_route_out(out, qbar, B * H, M)
     row_ptr, col_idx, nnz, row_max = out
     _check("psa_route_thresh", lib().psa_route_thresh(
         _ptr(qbar), _ptr(kbar), B, H, M, d, float(alpha), int(causal), int(keep_first), _ptr(row_ptr),
@@ -179,11 +228,13 @@ def psa_route_thresh_prob(qbar, kbar, alpha: float, causal: bool = False, keep_f
                           ws=None, capacity: int | None = None, out=None, stream=None):
     """Threshold routing in the probability domain: keep J iff
     s_IJ >= max_J s_IJ + ln(alpha).  Returns (row_ptr, col_idx, nnz, row_max)."""
-    B, H, M, d = (int(x) for x in qbar.shape)
+    B, H, M, d = _expect_stats(qbar, kbar)
     if ws is None:
         ws = workspace(B, H, M * 64, d, qbar.device)
     if out is None:
         out = _route_out(B, H, M, causal, capacity, qbar.device)
+    _expect_ws(ws, qbar, B, H, M * 64, d)
+    _expect_route_out(out, qbar, B * H, M)
     row_ptr, col_idx, nnz, row_max = out
     _check("psa_route_thresh_prob", lib().psa_route_thresh_prob(
         _ptr(qbar), _ptr(kbar), B, H, M, d, float(alpha), int(causal), int(keep_first), _ptr(row_ptr),
@@ -191,18 +242,31 @@ def psa_route_thresh_prob(qbar, kbar, alpha: float, causal: bool = False, keep_f
     return row_ptr, col_idx, nnz, row_max
 
 
+def _expect_attn_inputs(q, kbar, vsum, row_ptr, col_idx, row_max, B, H, M, d):
+    _expect("kbar", kbar, q, (B, H, M, d), torch.float32)
+    _expect("vsum", vsum, q, (B, H, M, d), torch.float32)
+    _expect("row_ptr", row_ptr, q, dtype=torch.int32, min_numel=B * H * M + 1)
+    _expect("col_idx", col_idx, q, dtype=torch.int32, min_numel=1)
+    _expect("row_max", row_max, q, dtype=torch.float32, min_numel=B * H * M)
+
+
 def psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_size: int = 64,
              ws=None, out=None, lse=None, want_lse: bool = False, row_max=None, stream=None):
     """Returns out (bf16 [B,H,N,d]) and, if requested, lse (float32 [B,H,N]).
     ``row_max`` (optional) is a router's row maxima, used as the softmax
     stabiliser instead of computing it in the kernel."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _expect_qkv(q, k, v)
+    M = N // block_size if block_size > 0 else 0
+    _expect_attn_inputs(q, kbar, vsum, row_ptr, col_idx, row_max, B, H, M, d)
     if ws is None:
         ws = workspace(B, H, N, d, q.device)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    _expect_ws(ws, q, B, H, N, d)
+    _expect("out", out, q, (B, H, N, d), torch.bfloat16)
+    _expect("lse", lse, q, (B, H, N), torch.float32)
     _check("psa_attn", lib().psa_attn(
         _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
         _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
@@ -213,13 +277,16 @@ def psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_
 def psa_dense(q, k, v, causal: bool = False, ws=None, out=None, lse=None, want_lse: bool = False,
               stream=None):
     """Dense softmax attention through the same tensor-core kernel."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _expect_qkv(q, k, v)
     if ws is None:
         ws = workspace(B, H, N, d, q.device)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    _expect_ws(ws, q, B, H, N, d)
+    _expect("out", out, q, (B, H, N, d), torch.bfloat16)
+    _expect("lse", lse, q, (B, H, N), torch.float32)
     _check("psa_dense", lib().psa_dense(
         _ptr(q), _ptr(k), _ptr(v), B, H, N, d, int(causal), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
         _stream(stream)))
@@ -233,9 +300,14 @@ def psa_attn_noalloc(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False
     that forbid allocation after start-up): the library's own 16 MiB scratch
     array is used instead, and calls that overlap on the GPU race on it.  ``status`` is an optional device
     int32 tensor that receives this call's device status word."""
-    B, H, N, d = _shape(q)
+    B, H, N, d = _expect_qkv(q, k, v)
+    M = N // block_size if block_size > 0 else 0
+    _expect_attn_inputs(q, kbar, vsum, row_ptr, col_idx, row_max, B, H, M, d)
     if out is None:
         out = torch.empty_like(q)
+    _expect("out", out, q, (B, H, N, d), torch.bfloat16)
+    _expect("lse", lse, q, (B, H, N), torch.float32)
+    _expect("status", status, q, dtype=torch.int32, min_numel=1)
     _check("psa_attn_noalloc", lib().psa_attn_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
         _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(status),
@@ -251,6 +323,7 @@ def psa_test_stall_next_attn(on: bool = True) -> None:
 
 def psa_read_status(ws, stream=None) -> int:
     """Synchronise the stream and return the device status word of ``ws``."""
+    _expect("ws", ws, dtype=torch.uint8, min_numel=256)
     st = ctypes.c_int(-1)
     _check("psa_read_status", lib().psa_read_status(_ptr(ws), ctypes.byref(st), _stream(stream)))
     return int(st.value)
