@@ -417,6 +417,10 @@ def gpu_arm(args):
                     "pool_gbs": None if st.dense else round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3) / 1e9, 1),
                     "pool_hbm_frac": None if st.dense else round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3)
                                                                  / 1e9 / peaks["hbm_gbs"], 4),
+                    # pool and route as one pass over the pooled inputs' HBM bytes (the
+                    # routing itself reads only the pooled statistics)
+                    "pool_route_hbm_frac": None if st.dense else round(
+                        pool_bytes(st.B, st.H, st.N, st.d) / ((pool_avg + route_avg) * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                     "attn_executed_tflops": round(achieved, 2),
                     "attn_effective_tflops": round(de_flops / (attn_avg * 1e-3) / 1e12, 2)},
         "flops": {"dense_equivalent": de_flops, "executed": ex_flops, "mma_issued": is_flops,
