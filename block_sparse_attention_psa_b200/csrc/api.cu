@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "internal.h"
@@ -78,6 +79,29 @@ int device_sm_count() {
   return n;
 }
 
+// The current device must be an sm_100 part, and the memory each pointer
+// names must live on it: a kernel launched on the current device would
+// otherwise address another GPU's memory (or host memory) through its TMA
+// descriptors and bulk stores.  Host and unregistered memory is rejected.
+int check_device_pointers(std::initializer_list<const void*> ptrs) {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PSA_ERR_DEVICE;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return PSA_ERR_DEVICE;
+  if (major != 10) return PSA_ERR_DEVICE;
+  for (const void* p : ptrs) {
+    if (!p) continue;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      cudaGetLastError();  // clear the sticky-free error of the query
+      return PSA_ERR_ARG;
+    }
+    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) return PSA_ERR_ARG;
+    if (at.type == cudaMemoryTypeDevice && at.device != dev) return PSA_ERR_DEVICE;
+  }
+  return PSA_OK;
+}
+
 std::atomic<int> g_stall_request{0};
 
 int take_stall_request() { return g_stall_request.exchange(0); }
@@ -101,13 +125,7 @@ int check_shape(int B, int H, int N, int d, int block_size) {
   return PSA_OK;
 }
 
-int check_device() {
-  int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PSA_ERR_DEVICE;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-    return PSA_ERR_DEVICE;
-  return major == 10 ? PSA_OK : PSA_ERR_DEVICE;
-}
+int check_device(std::initializer_list<const void*> ptrs) { return psa::check_device_pointers(ptrs); }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? PSA_OK : PSA_ERR_CUDA; }
 
@@ -145,7 +163,7 @@ int route_thresh_common(const float* qbar, const float* kbar, int B, int H, int 
   const long long bh = static_cast<long long>(B) * H;
   const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
   if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
-  if ((s = check_device()) != PSA_OK) return s;
+  if ((s = check_device({qbar, row_ptr, workspace})) != PSA_OK) return s;
   const long long cap = capacity > static_cast<size_t>(INT_MAX) ? INT_MAX : static_cast<long long>(capacity);
   char* ws = static_cast<char*>(workspace);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -171,7 +189,7 @@ const char* psa_status_string(int status) {
     case PSA_ERR_CUDA: return "a CUDA runtime call failed";
     case PSA_ERR_TIMEOUT: return "device: a bounded wait ran out and the kernel stopped";
     case PSA_ERR_CSR: return "device: a block list entry was out of range or repeated";
-    case PSA_ERR_DEVICE: return "no sm_100 (B200) device is current";
+    case PSA_ERR_DEVICE: return "no sm_100 (B200) device is current, or a tensor lives on another device";
     default: return "unknown status";
   }
 }
@@ -197,7 +215,7 @@ int psa_pool(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qbar) || !aligned16(kbar) ||
       !aligned16(vsum))
     return PSA_ERR_ARG;
-  if ((s = check_device()) != PSA_OK) return s;
+  if ((s = check_device({q, qbar})) != PSA_OK) return s;
   return cuda_status(psa::launch_pool(q, k, v, B * H, N / kBlock, d, qbar, kbar, vsum,
                                       static_cast<cudaStream_t>(stream)));
 }
@@ -223,7 +241,7 @@ int psa_route_topk(const float* qbar, const float* kbar, int B, int H, int M, in
   if (total > INT_MAX || static_cast<size_t>(total) > capacity) return PSA_ERR_CAPACITY;
   const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
   if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
-  if ((s = check_device()) != PSA_OK) return s;
+  if ((s = check_device({qbar, row_ptr, workspace})) != PSA_OK) return s;
   char* ws = static_cast<char*>(workspace);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
@@ -265,7 +283,7 @@ int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, cons
   const int M = N / kBlock;
   const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
   if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
-  if ((s = check_device()) != PSA_OK) return s;
+  if ((s = check_device({q, out, workspace})) != PSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
@@ -314,7 +332,7 @@ int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int
   const int M = N / kBlock;
   const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
   if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
-  if ((s = check_device()) != PSA_OK) return s;
+  if ((s = check_device({q, out, workspace})) != PSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
@@ -346,6 +364,17 @@ int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int
 int psa_test_stall_next_attn(int on) {
   if (on != 0 && on != 1) return PSA_ERR_ARG;
   psa::g_stall_request.store(on);
+  return PSA_OK;
+}
+
+int psa_read_fixup_count(const void* workspace, int* count, void* stream) {
+  if (!workspace || !count) return PSA_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, static_cast<const int*>(workspace) + 1, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return PSA_ERR_CUDA;
+  *count = v;
   return PSA_OK;
 }
 

@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <initializer_list>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -99,5 +100,8 @@ int take_stall_request();
 CUresult encode_tensor_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
                                    uint64_t outer, uint32_t box_inner, uint32_t box_rows);
 int device_sm_count();
+// PSA_OK if the current device is sm_100 and every non-null pointer names
+// device (or managed) memory of that device; else PSA_ERR_DEVICE / PSA_ERR_ARG.
+int check_device_pointers(std::initializer_list<const void*> ptrs);
 
 }  // namespace psa

@@ -28,7 +28,11 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
+// per device: the device address of the array in the context it was looked
+// up in, and that context's unique id (ids are never reused, so a reset
+// device, whose next context reloads the module, is set up again)
 void* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -38,17 +42,48 @@ size_t scratch_bytes(long long BH, long long M, long long d) {
   return 256 + align256(static_cast<size_t>(BH * M) * 4) + 2 * align256(static_cast<size_t>(BH * M * d) * 2);
 }
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the current device's context (0 if it cannot be read).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 // Device address of the scratch array on the current device.  The host-side
-// symbol is only a stand-in, never a device address: it is looked up once
-// per device, with that device current, and cached.
+// symbol is only a stand-in, never a device address: the address is looked up
+// with the device current, once per device context (the first call on a
+// device, and the first after a device reset), and cached.
 int scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PSA_ERR_DEVICE;
+  // the device's primary context, current on this thread (cudaSetDevice
+  // initialises it, so the context id below is the one kernels run in)
+  if (cudaSetDevice(dev) != cudaSuccess) return PSA_ERR_DEVICE;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || ctx == 0 || g_scratch_ctx[dev] != ctx) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return PSA_ERR_CUDA;
     g_scratch_ptr[dev] = ptr;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return PSA_OK;
@@ -78,12 +113,10 @@ int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
   const long long bh = static_cast<long long>(B) * H;
   const int M = N / psa::kBlock;
   if (scratch_bytes(bh, M, d) > kNoAllocScratchBytes) return PSA_ERR_CAPACITY;  // shape too large
-  int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10)
-    return PSA_ERR_DEVICE;
+  int s = psa::check_device_pointers({q, out});
+  if (s != PSA_OK) return s;
   void* base = nullptr;
-  int s = scratch_for_current_device(&base);
+  s = scratch_for_current_device(&base);
   if (s != PSA_OK) return s;
   char* ws = static_cast<char*>(base);
   const size_t off_fix = 256;

@@ -10,12 +10,13 @@
 //
 // A CTA of 256 threads copies the score rows of R consecutive query blocks
 // of one head into shared memory, and then one warp per row selects.  Top-k
-// finds the k-th largest score exactly by a 32-step bitwise search over the
-// order-preserving integer image of the fp32 scores (ties resolved by
-// ascending J), so it needs no sort; both routers write the list in
-// ascending J with warp ballots, and, when asked, each row's largest
-// candidate score (the attention step's softmax stabiliser).  Heads are
-// routed in batches whose score matrices fit the workspace.
+// finds the k-th largest score exactly by a radix select over the four 8-bit
+// digits of the order-preserving integer image of the fp32 scores (one
+// 256-bucket warp histogram per digit; ties resolved by ascending J), so it
+// needs no sort; both routers write the list in ascending J with warp
+// ballots, and, when asked, each row's largest candidate score (the
+// attention step's softmax stabiliser).  Heads are routed in batches whose
+// score matrices fit the workspace.
 #include "internal.h"
 #include "sm100.cuh"
 

@@ -14,6 +14,11 @@ round-to-nearest-even):
   centroid + 0.3 * N(0, I_d); four distinct key blocks per head, chosen
   uniformly, have their key centroid scaled by 3 (vertical stripes);
   V ~ N(0, 1).
+* ``clustered_wide``: as ``clustered`` with both centroids scaled by 4 and
+  token noise N(0, 1): block scores reach ~170 and a query's logits spread
+  ~+-50 around its block's score, so the per-block softmax stabiliser of the
+  attention kernel is far from some rows' largest terms (a stress input for
+  its exact fixup path).
 * ``clustered_slash``: as ``clustered``, and before the x3 scaling each query
   centroid I >= 8 gets (2 / sqrt(d)) * cK_{I-8} added, which raises the
   expected block score of the pair (I, I-8) by about 2 (a slash pattern).
@@ -50,6 +55,10 @@ WORKLOADS = {
     "dit_video_n32k_thresh_prob": dict(B=1, H=12, N=32768, d=128, gen="clustered",
                                        causal=False, routing=("thresh_prob", 0.5),
                                        keep_first=False),
+    # DiT-video shaped with wide logits (centroids x4, token noise 1): the
+    # fixed per-block softmax stabiliser misses some rows by > 2^60
+    "dit_video_n32k_wide": dict(B=1, H=12, N=32768, d=128, gen="clustered_wide",
+                                causal=False, routing=("topk", 0.15), keep_first=False),
     # long causal prefill, threshold 0.5, block 0 and diagonal always kept
     "long_causal_n128k": dict(B=1, H=8, N=131072, d=128, gen="clustered_slash",
                               causal=True, routing=("thresh", 0.5), keep_first=True),
@@ -80,17 +89,22 @@ def make_qkv(B: int, H: int, N: int, d: int, gen: str = "iid", seed: int = 0,
                 qh = rng.standard_normal((N, d), dtype=np.float32)
                 kh = rng.standard_normal((N, d), dtype=np.float32)
                 vh = rng.standard_normal((N, d), dtype=np.float32)
-            elif gen in ("clustered", "clustered_slash"):
+            elif gen in ("clustered", "clustered_slash", "clustered_wide"):
+                wide = gen == "clustered_wide"
+                cscale, noise = (np.float32(4.0), np.float32(1.0)) if wide else (np.float32(1.0), np.float32(0.3))
                 cq = rng.standard_normal((M, d), dtype=np.float32)
                 ck = rng.standard_normal((M, d), dtype=np.float32)
+                if wide:
+                    cq *= cscale
+                    ck *= cscale
                 heavy = rng.choice(M, size=min(4, M), replace=False)
                 if gen == "clustered_slash" and M > 8:
                     cq[8:] += np.float32(2.0 / math.sqrt(d)) * ck[:-8]
                 ck[heavy] *= np.float32(3.0)
                 qh = np.repeat(cq, block, axis=0)
-                qh += np.float32(0.3) * rng.standard_normal((N, d), dtype=np.float32)
+                qh += noise * rng.standard_normal((N, d), dtype=np.float32)
                 kh = np.repeat(ck, block, axis=0)
-                kh += np.float32(0.3) * rng.standard_normal((N, d), dtype=np.float32)
+                kh += noise * rng.standard_normal((N, d), dtype=np.float32)
                 vh = rng.standard_normal((N, d), dtype=np.float32)
             else:
                 raise ValueError(f"unknown generator {gen!r}")

@@ -3,7 +3,8 @@
 Argument marshalling only: every step runs in the library's CUDA kernels.
 Each function has the name of the C entry point it calls.  Tensors are
 PyTorch CUDA tensors (PyTorch is used for device memory and streams); the
-call is issued on ``torch.cuda.current_stream()`` unless a stream is given.
+call is issued with the device of its main tensor current, on that device's
+``torch.cuda.current_stream()`` unless a stream is given.
 A non-zero status raises :class:`PSAError`.  There is no fallback: if the
 library is missing, :func:`lib` raises.
 """
@@ -30,7 +31,8 @@ PSA_ERR_DEVICE = 8
 
 EXPORTS = ("psa_status_string", "psa_version", "psa_workspace_size", "psa_route_capacity", "psa_pool",
            "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense", "psa_read_status",
-           "psa_attn_noalloc", "psa_route_thresh_prob", "psa_test_stall_next_attn")
+           "psa_attn_noalloc", "psa_route_thresh_prob", "psa_test_stall_next_attn",
+           "psa_read_fixup_count")
 
 _lib = None
 
@@ -55,6 +57,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "psa_attn": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, Z, P]),
         "psa_dense": (I, [P, P, P, I, I, I, I, I, P, P, P, Z, P]),
         "psa_read_status": (I, [P, ctypes.POINTER(I), P]),
+        "psa_read_fixup_count": (I, [P, ctypes.POINTER(I), P]),
         "psa_test_stall_next_attn": (I, [I]),
         "psa_attn_noalloc": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, P]),
     }
@@ -96,9 +99,20 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    s = stream if stream is not None else torch.cuda.current_stream()
+def _stream(stream, like):
+    """The caller's stream, else the current stream of the problem's device."""
+    s = stream if stream is not None else torch.cuda.current_stream(like.device)
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _call(fn: str, like, *args) -> None:
+    """Call the C entry point with the device of ``like`` (the problem's main
+    tensor) current: the library launches on the current device and sizes its
+    TMA descriptors and scratch for it, so the tensors' device must be the
+    current one (the library itself refuses a mismatch with PSA_ERR_DEVICE)."""
+    with torch.cuda.device(like.device):
+        status = getattr(lib(), fn)(*args)
+    _check(fn, status)
 
 
 def _shape(q):
@@ -168,8 +182,8 @@ def psa_pool(q, k, v, block_size: int = 64, out=None, stream=None):
     qbar, kbar, vsum = out
     for name, t in (("qbar", qbar), ("kbar", kbar), ("vsum", vsum)):
         _expect(name, t, q, (B, H, M, d), torch.float32)
-    _check("psa_pool", lib().psa_pool(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, block_size,
-                                      _ptr(qbar), _ptr(kbar), _ptr(vsum), _stream(stream)))
+    _call("psa_pool", q, _ptr(q), _ptr(k), _ptr(v), B, H, N, d, block_size,
+          _ptr(qbar), _ptr(kbar), _ptr(vsum), _stream(stream, q))
     return qbar, kbar, vsum
 
 
@@ -201,9 +215,9 @@ def psa_route_topk(qbar, kbar, density: float, causal: bool = False, capacity: i
     _expect_ws(ws, qbar, B, H, M * 64, d)
     _expect_route_out(out, qbar, B * H, M)
     row_ptr, col_idx, nnz, row_max = out
-    _check("psa_route_topk", lib().psa_route_topk(
-        _ptr(qbar), _ptr(kbar), B, H, M, d, float(density), int(causal), _ptr(row_ptr), _ptr(col_idx),
-        col_idx.numel(), _ptr(nnz), _ptr(row_max), _ptr(ws), ws.numel(), _stream(stream)))
+    _call("psa_route_topk", qbar, _ptr(qbar), _ptr(kbar), B, H, M, d, float(density), int(causal),
+          _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(row_max), _ptr(ws), ws.numel(),
+          _stream(stream, qbar))
     return row_ptr, col_idx, nnz, row_max
 
 
@@ -218,9 +232,9 @@ def psa_route_thresh(qbar, kbar, alpha: float, causal: bool = False, keep_first:
     _expect_ws(ws, qbar, B, H, M * 64, d)
     _expect_route_out(out, qbar, B * H, M)
     row_ptr, col_idx, nnz, row_max = out
-    _check("psa_route_thresh", lib().psa_route_thresh(
-        _ptr(qbar), _ptr(kbar), B, H, M, d, float(alpha), int(causal), int(keep_first), _ptr(row_ptr),
-        _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(row_max), _ptr(ws), ws.numel(), _stream(stream)))
+    _call("psa_route_thresh", qbar, _ptr(qbar), _ptr(kbar), B, H, M, d, float(alpha), int(causal),
+          int(keep_first), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(row_max), _ptr(ws),
+          ws.numel(), _stream(stream, qbar))
     return row_ptr, col_idx, nnz, row_max
 
 
@@ -236,9 +250,9 @@ def psa_route_thresh_prob(qbar, kbar, alpha: float, causal: bool = False, keep_f
     _expect_ws(ws, qbar, B, H, M * 64, d)
     _expect_route_out(out, qbar, B * H, M)
     row_ptr, col_idx, nnz, row_max = out
-    _check("psa_route_thresh_prob", lib().psa_route_thresh_prob(
-        _ptr(qbar), _ptr(kbar), B, H, M, d, float(alpha), int(causal), int(keep_first), _ptr(row_ptr),
-        _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(row_max), _ptr(ws), ws.numel(), _stream(stream)))
+    _call("psa_route_thresh_prob", qbar, _ptr(qbar), _ptr(kbar), B, H, M, d, float(alpha), int(causal),
+          int(keep_first), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(row_max), _ptr(ws),
+          ws.numel(), _stream(stream, qbar))
     return row_ptr, col_idx, nnz, row_max
 
 
@@ -267,10 +281,9 @@ def psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_
     _expect_ws(ws, q, B, H, N, d)
     _expect("out", out, q, (B, H, N, d), torch.bfloat16)
     _expect("lse", lse, q, (B, H, N), torch.float32)
-    _check("psa_attn", lib().psa_attn(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
-        _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
-        _stream(stream)))
+    _call("psa_attn", q, _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx),
+          col_idx.numel(), _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(ws),
+          ws.numel(), _stream(stream, q))
     return (out, lse) if lse is not None else out
 
 
@@ -287,9 +300,8 @@ def psa_dense(q, k, v, causal: bool = False, ws=None, out=None, lse=None, want_l
     _expect_ws(ws, q, B, H, N, d)
     _expect("out", out, q, (B, H, N, d), torch.bfloat16)
     _expect("lse", lse, q, (B, H, N), torch.float32)
-    _check("psa_dense", lib().psa_dense(
-        _ptr(q), _ptr(k), _ptr(v), B, H, N, d, int(causal), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
-        _stream(stream)))
+    _call("psa_dense", q, _ptr(q), _ptr(k), _ptr(v), B, H, N, d, int(causal), _ptr(out), _ptr(lse), _ptr(ws),
+          ws.numel(), _stream(stream, q))
     return (out, lse) if lse is not None else out
 
 
@@ -308,10 +320,9 @@ def psa_attn_noalloc(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False
     _expect("out", out, q, (B, H, N, d), torch.bfloat16)
     _expect("lse", lse, q, (B, H, N), torch.float32)
     _expect("status", status, q, dtype=torch.int32, min_numel=1)
-    _check("psa_attn_noalloc", lib().psa_attn_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
-        _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(status),
-        _stream(stream)))
+    _call("psa_attn_noalloc", q, _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr),
+          _ptr(col_idx), col_idx.numel(), _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out),
+          _ptr(lse), _ptr(status), _stream(stream, q))
     return out
 
 
@@ -325,8 +336,17 @@ def psa_read_status(ws, stream=None) -> int:
     """Synchronise the stream and return the device status word of ``ws``."""
     _expect("ws", ws, dtype=torch.uint8, min_numel=256)
     st = ctypes.c_int(-1)
-    _check("psa_read_status", lib().psa_read_status(_ptr(ws), ctypes.byref(st), _stream(stream)))
+    _call("psa_read_status", ws, _ptr(ws), ctypes.byref(st), _stream(stream, ws))
     return int(st.value)
+
+
+def psa_read_fixup_count(ws, stream=None) -> int:
+    """Synchronise the stream and return how many query blocks the last
+    attention call on ``ws`` recomputed through its exact fixup path."""
+    _expect("ws", ws, dtype=torch.uint8, min_numel=256)
+    n = ctypes.c_int(-1)
+    _call("psa_read_fixup_count", ws, _ptr(ws), ctypes.byref(n), _stream(stream, ws))
+    return int(n.value)
 
 
 def psa_forward(q, k, v, mode: str = "topk", density: float = 0.15, alpha: float = 0.5,

@@ -14,7 +14,10 @@
  *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL = the legacy default stream) and returns a status code.
  *  - Arguments are validated on the host before any launch: a bad argument
- *    returns an error code and launches nothing.  Conditions that only the
+ *    returns an error code and launches nothing.  The tensors must live on
+ *    the CURRENT device (cudaSetDevice): a call whose main input or output
+ *    is memory of another device returns PSA_ERR_DEVICE, one given host
+ *    memory returns PSA_ERR_ARG.  Conditions that only the
  *    device can see (a malformed block list, a bounded wait that ran out) are
  *    recorded in the status word inside the caller's workspace; read it with
  *    psa_read_status().
@@ -54,7 +57,7 @@ enum psa_status {
     PSA_ERR_CUDA = 5,         /* a CUDA runtime / driver call failed           */
     PSA_ERR_TIMEOUT = 6,      /* device: a bounded wait ran out (kernel quit)   */
     PSA_ERR_CSR = 7,          /* device: a listed block is out of range or repeated */
-    PSA_ERR_DEVICE = 8        /* no sm_100 device current                      */
+    PSA_ERR_DEVICE = 8        /* no sm_100 device current, or a tensor of another device */
 };
 
 /* Text for a status code (static storage, never NULL). */
@@ -218,8 +221,10 @@ PSA_API int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t
  * fixup list) lives in a 16 MiB array inside the library, so shapes need
  * 256 + 4*B*H*M + 4*B*H*M*d bytes (each part rounded up to 256 bytes) to fit
  * in 16 MiB, else PSA_ERR_CAPACITY.  The first call on a device looks up the
- * array's device address (make it before any stream capture).  Every call on
- * a device shares the array: calls whose work overlaps on the GPU race.
+ * array's device address (make it before any stream capture); so does the
+ * first call after a device reset, which loads the library's device code
+ * anew.  Every call on a device shares the array: calls whose work overlaps
+ * on the GPU race.
  * `status` (device int, nullable) receives the device status word of this
  * call (PSA_OK, PSA_ERR_CSR or PSA_ERR_TIMEOUT) in stream order.  Never
  * allocates device memory.
@@ -248,6 +253,17 @@ PSA_API int psa_test_stall_next_attn(int on);
  * psa_dense reset it at their start).  Returns PSA_OK or PSA_ERR_CUDA.
  */
 PSA_API int psa_read_status(const void* workspace, int* status, void* stream);
+
+/*
+ * Synchronises `stream`, then copies into *count (host pointer) the number of
+ * query blocks (64 rows each) that the last psa_attn / psa_dense call on
+ * `workspace` recomputed through its exact fixup path: the blocks with a row
+ * whose softmax denominator, under the kernel's fixed per-block stabiliser,
+ * left [2^-60, 2^60] (an implementation detail with no counterpart in the
+ * method's sources; it measures how often the slow path ran).  Returns
+ * PSA_OK or PSA_ERR_CUDA.
+ */
+PSA_API int psa_read_fixup_count(const void* workspace, int* count, void* stream);
 
 #ifdef __cplusplus
 }

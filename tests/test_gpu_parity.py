@@ -27,6 +27,27 @@ def _full_check(q, k, v, mode, param, causal=False, keep_first=False, units=None
     return check_output(g, q, k, v, kbar, vsum, causal, units)
 
 
+def _routed_full_check(q, k, v, mode, param, causal=False, keep_first=False, units=None):
+    """As _full_check, returning the GPU results."""
+    g = run_gpu(q, k, v, mode, param, causal, keep_first)
+    assert g["status"] == psa.PSA_OK, psa.status_text(g["status"])
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    check_routing(g, O.block_scores(qbar, kbar), mode, param, causal, keep_first)
+    check_output(g, q, k, v, kbar, vsum, causal, units)
+    return g
+
+
+_INPUTS = {}
+
+
+def _workload_inputs(name):
+    """The workload's tensors, generated once per test session."""
+    if name not in _INPUTS:
+        _INPUTS.clear()
+        _INPUTS[name] = workload_inputs(name)
+    return _INPUTS[name]
+
+
 # ------------------------------------------------------------------ small, every unit
 def test_tiny_iid_topk_quarter():
     q, k, v = workload_inputs("tiny_iid_n1k")
@@ -107,13 +128,25 @@ def test_dense_equals_softmax_attention(d, causal):
     assert np.abs(f64(lse) - ref_lse).max() <= 1e-3 * max(1.0, np.abs(ref_lse).max())
 
 
-def test_tiny_density_one_equals_dense():
+def test_tiny_density_one_against_oracle_and_softmax():
+    # the tiny i.i.d. workload at density 1 on its own tensors: every block is
+    # listed, so the routed path and psa_dense must both equal the oracle (fed
+    # the GPU's lists) and textbook softmax attention (fp64 SDPA)
     q, k, v = workload_inputs("tiny_iid_n1k")
-    g = run_gpu(q, k, v, "topk", 1.0)
+    B, H, N, d = q.shape
+    M = N // 64
+    g = _routed_full_check(q, k, v, "topk", 1.0)
+    assert np.array_equal(np.diff(g["row_ptr"]), np.full(B * H * M, M))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(f64(q)), torch.from_numpy(f64(k)), torch.from_numpy(f64(v))).numpy()
     dq, dk, dv = (x.cuda() for x in (q, k, v))
-    dense = psa.psa_dense(dq, dk, dv, False)
-    err = np.abs(f64(g["out"]) - f64(dense))
-    assert err.max() <= 2e-2 and err.mean() <= 2e-3
+    dense, dense_lse = psa.psa_dense(dq, dk, dv, False, want_lse=True)
+    for got in (f64(g["out"]), f64(dense)):
+        err = np.abs(got - ref)
+        assert err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
+    gd = dict(out=dense.cpu(), lse=dense_lse.cpu(), row_ptr=g["row_ptr"], col_idx=g["col_idx"], status=psa.PSA_OK)
+    _, kbar, vsum = O.pool(f64(q), f64(k), f64(v))
+    check_output(gd, q, k, v, kbar, vsum, False)
 
 
 # ------------------------------------------------------------------ hand-built block lists
@@ -193,7 +226,7 @@ def test_huge_logit_goes_through_exact_fixup():
 # ------------------------------------------------------------------ full-size workloads
 def _full_size(name, density=None, n_units=48):
     w = WORKLOADS[name]
-    q, k, v = workload_inputs(name)
+    q, k, v = _workload_inputs(name)
     mode, param = w["routing"]
     if density is not None:
         param = density
@@ -232,8 +265,10 @@ def test_full_long_causal_threshold():
     _full_size("long_causal_n128k", n_units=40)
 
 
-@pytest.mark.parametrize("density", [0.05, 1.0])
+@pytest.mark.parametrize("density", [0.05, 0.10, 0.15, 0.30, 1.0])
 def test_full_sweep(density):
+    # every density of the d = 64 sweep, routed and attended exactly as the
+    # bench runs it
     _full_size("sweep_n64k", density=density, n_units=40)
 
 
@@ -299,8 +334,9 @@ def test_maximum_block_count():
 
 @pytest.mark.parametrize("M,causal", [(1024, False), (1024, True), (1100, False), (1100, True)])
 def test_topk_selection_on_both_sides_of_1024_candidates(M, causal):
-    # rows of up to 1024 candidates are selected with their keys in registers,
-    # longer rows from shared memory: both against the oracle on every row
+    # rows of 1024 and 1100 candidates (the radix select's histograms and the
+    # ballot passes over more than 32 words of candidates), causal and not,
+    # against the oracle on every row
     q, k, v = make_qkv(1, 2, M * 64, 64, "clustered", seed=23)
     g = run_gpu(q, k, v, "topk", 0.1, causal)
     assert g["status"] == psa.PSA_OK
@@ -401,3 +437,85 @@ def test_full_size_dense_sampled(name):
     g = dict(out=out.cpu(), lse=lse.cpu(), row_ptr=rp, col_idx=ci, status=status)
     _, kb, vs = O.pool(f64(q), f64(k), f64(v))
     check_output(g, q, k, v, kb, vs, causal, sample_units(B, H, M, 16, seed=9))
+
+
+# ------------------------------------------------------------------ rows longer than the cached list
+@pytest.mark.parametrize("causal", [False, True])
+def test_topk_rows_of_more_than_1024_listed_blocks(causal):
+    # M = 1536 at density 0.8: k = ceil(fl32(0.8) * 1536) = 1229 listed blocks
+    # per row (causal: every row with I >= 1228), more than the 1024 entries
+    # the attention kernel keeps in shared memory, so the tail of each list is
+    # read from global memory
+    M, d = 1536, 64
+    q, k, v = make_qkv(1, 1, M * 64, d, "clustered", seed=26)
+    g = run_gpu(q, k, v, "topk", 0.8, causal)
+    assert g["status"] == psa.PSA_OK
+    assert np.diff(g["row_ptr"]).max() == 1229
+    qbar, kbar, vsum = check_pool(g, q, k, v)
+    check_routing(g, O.block_scores(qbar, kbar), "topk", 0.8, causal)
+    units = [(0, 0, I) for I in (0, 700, 1228, 1229, 1400, M - 1)]
+    check_output(g, q, k, v, kbar, vsum, causal, units)
+
+
+def test_hand_built_rows_of_1100_to_2000_blocks():
+    # M = 2048, d = 128: rows listing 1100 to 2000 random blocks (and a few
+    # short ones), against the oracle fed the same lists
+    rng = np.random.default_rng(27)
+    M, d = 2048, 128
+    q, k, v = make_qkv(1, 1, M * 64, d, "clustered", seed=27)
+    lists = []
+    for I in range(M):
+        n = int(rng.integers(1100, 2001)) if I % 3 else int(rng.integers(0, 40))
+        lists.append(np.sort(rng.choice(M, size=n, replace=False)))
+    g = _attn_with_lists(q, k, v, lists, False)
+    assert g["status"] == psa.PSA_OK
+    _, kbar, vsum = O.pool(f64(q), f64(k), f64(v))
+    units = [(0, 0, I) for I in (1, 2, 3, 1024, 2047)]
+    check_output(g, q, k, v, kbar, vsum, False, units)
+
+
+# ------------------------------------------------------------------ boundary: where the tensors live
+def test_host_memory_is_refused_before_any_launch():
+    # the library takes device pointers of the current device only: host
+    # memory (pageable or pinned) is refused on the host with PSA_ERR_ARG
+    L = psa.lib()
+    B, H, N, d = 1, 1, 128, 64
+    M = N // 64
+    dev = [torch.zeros(B, H, N, d, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    stats = [torch.zeros(B, H, M, d, device="cuda") for _ in range(3)]
+    pinned = torch.zeros(B, H, N, d, dtype=torch.bfloat16).pin_memory()
+    pageable = np.zeros(B * H * N * d + 8, dtype=np.uint16)
+    host_ptr = pageable.ctypes.data + (-pageable.ctypes.data) % 16
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    for bad in (ctypes.c_void_p(pinned.data_ptr()), ctypes.c_void_p(host_ptr)):
+        rc = L.psa_pool(bad, P(dev[1]), P(dev[2]), B, H, N, d, 64, *(P(t) for t in stats), None)
+        assert rc == psa.PSA_ERR_ARG, psa.status_text(rc)
+    # the same call on device memory runs
+    rc = L.psa_pool(*(P(t) for t in dev), B, H, N, d, 64, *(P(t) for t in stats), None)
+    assert rc == psa.PSA_OK
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ wide logits: the exact fixup path
+def test_wide_logits_small_every_unit():
+    # centroids x4, token noise 1: some query rows' logits sit far above their
+    # block's stabiliser, so their blocks go through the fixup path; every
+    # unit against the oracle, and the fixup count is reported
+    q, k, v = make_qkv(1, 2, 96 * 64, 128, "clustered_wide", seed=28)
+    dq, dk, dv = (x.cuda() for x in (q, k, v))
+    B, H, N, d = q.shape
+    ws = psa.workspace(B, H, N, d)
+    qbar, kbar, vsum = psa.psa_pool(dq, dk, dv)
+    rp, ci, nnz, row_max = psa.psa_route_topk(qbar, kbar, 0.15, ws=ws)
+    out, lse = psa.psa_attn(dq, dk, dv, kbar, vsum, rp, ci, ws=ws, row_max=row_max, want_lse=True)
+    fixed = psa.psa_read_fixup_count(ws)
+    assert 0 < fixed < B * H * (N // 64), fixed
+    n = int(nnz.item())
+    g = dict(out=out.cpu(), lse=lse.cpu(), row_ptr=rp.cpu().long().numpy(), col_idx=ci[:n].cpu().long().numpy(),
+             status=psa.psa_read_status(ws))
+    _, kb, vs = O.pool(f64(q), f64(k), f64(v))
+    check_output(g, q, k, v, kb, vs, False)
+
+
+def test_full_dit_video_wide_logits():
+    _full_size("dit_video_n32k_wide", n_units=40)

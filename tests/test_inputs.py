@@ -30,3 +30,12 @@ def test_workload_table():
     assert WORKLOADS["dit_video_n32k"]["N"] == 32768
     for w in WORKLOADS.values():
         assert w["N"] % 64 == 0 and w["d"] in (64, 128)
+
+
+def test_wide_structure():
+    q, k, v = make_qkv(1, 1, 64 * 32, 64, "clustered_wide", seed=0)
+    kb = k.float().reshape(32, 64, 64)
+    spread = (kb - kb.mean(1, keepdim=True)).std().item()
+    assert 0.9 < spread < 1.1
+    norms = kb.mean(1).norm(dim=-1)
+    assert (norms > 2 * 4 * np.sqrt(64)).sum().item() == 4
