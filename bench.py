@@ -152,10 +152,11 @@ class ClockSampler:
 class Step:
     """Device buffers and one step of the path for one workload."""
 
-    def __init__(self, name, density, seed, device, dense=False):
+    def __init__(self, name, density, seed, device, dense=False, hyd=False):
         w = dict(WORKLOADS[name])
         self.name = name
         self.dense = dense  # psa_dense (every candidate exact) instead of pool -> route -> attn
+        self.hyd = hyd      # first-order correction: + statistic, attention with the correction
         self.w = w
         self.B, self.H, self.N, self.d = w["B"], w["H"], w["N"], w["d"]
         self.M = self.N // 64
@@ -178,13 +179,15 @@ class Step:
         self.csr = (torch.empty(B * H * M + 1, **i32), torch.empty(cap, **i32), torch.empty(1, **i32),
                     torch.empty(B * H * M, dtype=torch.float32, device=device))
         self.ws = psa.workspace(B, H, self.N, d, device)
+        self.hstat = torch.empty(B, H, d, d, dtype=torch.float32, device=device)
         self.out = torch.empty_like(self.q)
         self.out_host = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
         self.stream = torch.cuda.current_stream()
-        self.launches = launches_per_step(B, H, self.M, self.mode, dense)
+        self.launches = launches_per_step(B, H, self.M, self.mode, dense, hyd)
 
     def run(self, ev=None, io=None, stream=None):
-        """pool -> route -> attention; ``ev`` = 4 events to split the kernels;
+        """pool -> route -> [statistic ->] attention; ``ev`` = 5 events to split
+        the kernels (pool | route | first-order statistic | attention);
         ``io`` = (q, k, v, out) device tensors (default: the step's own) and
         ``stream`` the stream to issue on (default: the current one)."""
         q, k, v, out = io if io is not None else (self.q, self.k, self.v, self.out)
@@ -195,9 +198,10 @@ class Step:
                 ev[0].record(s)
                 ev[1].record(s)
                 ev[2].record(s)
+                ev[3].record(s)
             psa.psa_dense(q, k, v, self.causal, ws=self.ws, out=out, stream=s)
             if ev:
-                ev[3].record(s)
+                ev[4].record(s)
             return
         if ev:
             ev[0].record(s)
@@ -215,10 +219,18 @@ class Step:
                                  out=self.csr, stream=s)
         if ev:
             ev[2].record(s)
-        psa.psa_attn(q, k, v, kbar, vsum, self.csr[0], self.csr[1], self.causal, ws=self.ws,
-                     out=out, row_max=self.csr[3], stream=s)
+        if self.hyd:
+            psa.psa_hyd_stat(k, v, kbar, vsum, ws=self.ws, out=self.hstat, stream=s)
         if ev:
             ev[3].record(s)
+        if self.hyd:
+            psa.psa_attn_hyd(q, k, v, kbar, vsum, self.hstat, self.csr[0], self.csr[1], self.causal, ws=self.ws,
+                             out=out, row_max=self.csr[3], stream=s)
+        else:
+            psa.psa_attn(q, k, v, kbar, vsum, self.csr[0], self.csr[1], self.causal, ws=self.ws,
+                         out=out, row_max=self.csr[3], stream=s)
+        if ev:
+            ev[4].record(s)
 
     def e2e_ms(self, nsteps):
         """Milliseconds per step with host buffers in and the host result out,
@@ -265,20 +277,22 @@ class Step:
         return self.out_host.numel() * self.out_host.element_size()
 
 
-def launches_per_step(B: int, H: int, M: int, mode: str, dense: bool) -> int:
-    """Kernels of ours one step launches: psa_dense = 3 (key pooling,
-    attention, fixup); otherwise pool 1, route = one split of both operands
-    plus, per batch of heads, one score and one selection launch (the library
-    batches as many heads as fit 256 MB of scores), plus scan and compaction
-    for the threshold routers, and attention 3 (bf16 statistics, attention,
-    fixup)."""
+def launches_per_step(B: int, H: int, M: int, mode: str, dense: bool, hyd: bool = False) -> int:
+    """Kernels of ours one step launches: psa_dense = 4 (key pooling,
+    attention, rerun of flagged blocks, exact fixup); otherwise pool 1, route
+    = one split of both operands plus, per batch of heads, one score and one
+    selection launch (the library batches as many heads as fit 256 MB of
+    scores), plus scan and compaction for the threshold routers, and attention
+    4 (bf16 statistics, attention, rerun of flagged blocks, exact fixup); the
+    first-order mode adds the statistic (2: partial sums and their reduction)
+    and the correction (1)."""
     if dense:
-        return 3
+        return 4
     Mp = -(-M // 128) * 128
     per_batch = max(1, min(B * H, (256 << 20) // (M * Mp * 4)))
     nb = -(-(B * H) // per_batch)
     route = 1 + 2 * nb + (0 if mode == "topk" else 2)
-    return 1 + route + 3
+    return 1 + route + 4 + (3 if hyd else 0)
 
 
 def _flush(buf):
@@ -331,7 +345,7 @@ def gpu_arm(args):
     if args.gpus != world and world > 1:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
     device = torch.device("cuda", local)
-    st = Step(args.workload, args.density, seed=rank, device=device, dense=args.dense)
+    st = Step(args.workload, args.density, seed=rank, device=device, dense=args.dense, hyd=args.hyd)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     for _ in range(args.warmup):
         st.run()
@@ -353,13 +367,17 @@ def gpu_arm(args):
         nnz = int(st.csr[2].item())
         ex_flops = executed_flops(rp, None, st.B, st.H, st.M, st.d, st.causal)
         is_flops = issued_flops(rp, st.B, st.H, st.M, st.d, st.causal)
+    # first-order mode: the correction X = Q H (2 N d^2 per head) in the
+    # attention call; the statistic (another 2 N d^2) is timed on its own
+    hyd_apply_flops = 2.0 * st.B * st.H * st.N * st.d * st.d if st.hyd else 0.0
+    ex_flops += hyd_apply_flops
     de_flops = dense_flops(st.B, st.H, st.N, st.d, st.causal)
     status = psa.psa_read_status(st.ws)
-    fixup_blocks = psa.psa_read_fixup_count(st.ws)
+    fixup_rerun, fixup_exact = psa.psa_read_fixup_count(st.ws)
 
     clocks = ClockSampler(local)
     clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     _barrier(world)
     torch.cuda.synchronize()
     for i in range(args.steps):
@@ -368,10 +386,11 @@ def gpu_arm(args):
     torch.cuda.synchronize()
     _barrier(world)
     clk = clocks.stop()
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
     pool_ms = [e[0].elapsed_time(e[1]) for e in evs]
     route_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    attn_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    stat_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    attn_ms = [e[3].elapsed_time(e[4]) for e in evs]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
 
@@ -384,6 +403,7 @@ def gpu_arm(args):
 
     peaks = _peaks()
     attn_avg = statistics.mean(attn_ms)
+    stat_avg = statistics.mean(stat_ms)
     pool_avg = statistics.mean(pool_ms)
     route_avg = statistics.mean(route_ms)
     achieved = ex_flops / (attn_avg * 1e-3) / 1e12
@@ -403,17 +423,22 @@ def gpu_arm(args):
         "data": "synthetic (seeded generator, seed = rank)",
         "config": {"workload": st.name, "B": st.B, "H": st.H, "N": st.N, "d": st.d, "block": 64,
                    "causal": st.causal, "routing": "dense (psa_dense)" if st.dense else f"{st.mode} {st.param}",
+                   "variant": "first-order (psa_hyd_stat + psa_attn_hyd)" if st.hyd else "0th-order (psa_attn)",
                    "keep_first": st.keep_first,
                    "parallelism": f"replicas x{world} (independent problems)" if world > 1 else "1 GPU",
                    "l2": "flushed between steps (512 MB write outside the timed events)"},
         "roofline": {"bound": "tensor",
-                     "kernel": "attn_kernel (psa_dense call)" if st.dense else "attn_kernel (psa_attn call)",
+                     "kernel": "attn_kernel (psa_dense call)" if st.dense else
+                     ("attn_kernel + hyd_apply_kernel (psa_attn_hyd call)" if st.hyd else "attn_kernel (psa_attn call)"),
                      "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": round(achieved / tc_peak, 4),
                      # the capture is of psa_attn at the workload's own routing
-                     "traffic": None if st.dense or args.density is not None else recorded_traffic(st.name),
+                     "traffic": None if st.dense or st.hyd or args.density is not None else recorded_traffic(st.name),
                      "peak_source": peaks["source"] + " bf16 burst"},
         "kernels": {"pool_ms": None if st.dense else round(pool_avg, 4),
+                    "hyd_stat_ms": round(stat_avg, 4) if st.hyd else None,
+                    "hyd_stat_gbs": round(2 * st.B * st.H * st.N * st.d * 2 / (stat_avg * 1e-3) / 1e9, 1)
+                    if st.hyd else None,
                     "route_ms": None if st.dense else round(route_avg, 4), "attn_ms": round(attn_avg, 4),
                     "pool_gbs": None if st.dense else round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3) / 1e9, 1),
                     "pool_hbm_frac": None if st.dense else round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3)
@@ -428,11 +453,12 @@ def gpu_arm(args):
                   "mma_issued_tflops": round(is_flops / (attn_avg * 1e-3) / 1e12, 2)},
         "density": {"realised": round(nnz / n_cand, 5), "listed_blocks": nnz},
         "device_status": status,
-        # query blocks of one step that the attention kernel's exact fixup path
-        # recomputed (rows whose denominator left [2^-60, 2^60] under the fixed
-        # per-block stabiliser); their cost is inside attn_ms
-        "fixup": {"query_blocks": fixup_blocks, "of": st.B * st.H * st.M,
-                  "share": round(fixup_blocks / (st.B * st.H * st.M), 6)},
+        # query blocks of one step whose denominator left [2^-60, 2^60] under the
+        # kernel's fixed per-block stabiliser: recomputed on the tensor cores with
+        # per-query stabilisers (rerun), and those that still needed the exact
+        # CUDA-core path; their cost is inside attn_ms
+        "fixup": {"rerun_blocks": fixup_rerun, "exact_blocks": fixup_exact, "of": st.B * st.H * st.M,
+                  "share": round(fixup_rerun / (st.B * st.H * st.M), 6)},
         "e2e": {"value": round(weak_scaling_value(de_flops, world, e2e_ms), 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": st.h2d_bytes(),
                 "d2h_bytes_per_step": st.d2h_bytes(), "steps": e2e_steps,
@@ -611,6 +637,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dense", action="store_true", help="time psa_dense (density 1, every block exact) instead")
+    ap.add_argument("--hyd", action="store_true",
+                    help="time the first-order variant (psa_hyd_stat + psa_attn_hyd) instead of psa_attn")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

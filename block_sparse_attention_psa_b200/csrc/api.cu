@@ -20,6 +20,10 @@ WorkspaceLayout workspace_layout(long long BH, long long M, long long d) {
   L.header = 0;
   L.fixup_list = o;
   o += align256(static_cast<size_t>(BH * M) * 4);
+  L.fixup_list2 = o;
+  o += align256(static_cast<size_t>(BH * M) * 4);
+  L.row_lse2 = o;
+  o += align256(static_cast<size_t>(BH * M * 64) * 4);
   L.kbar_bf16 = o;
   o += align256(static_cast<size_t>(BH * M * d) * 2);
   L.vsum_bf16 = o;
@@ -32,6 +36,10 @@ WorkspaceLayout workspace_layout(long long BH, long long M, long long d) {
   o += align256(static_cast<size_t>(3 * BH * M * d) * 2);
   L.k_split = o;
   o += align256(static_cast<size_t>(3 * BH * M * d) * 2);
+  L.hyd_w = o;
+  o += align256(static_cast<size_t>(BH * M * 64) * 4);
+  L.hyd_partial = o;
+  o += align256(psa::hyd_partial_bytes(static_cast<int>(BH), static_cast<int>(M), static_cast<int>(d)));
   // block scores of as many heads as fit 256 MB (at least one)
   const size_t head_scores = static_cast<size_t>(M) * score_stride(static_cast<int>(M)) * 4;
   const long long fit = static_cast<long long>((size_t(256) << 20) / head_scores);
@@ -175,6 +183,67 @@ int route_thresh_common(const float* qbar, const float* kbar, int B, int H, int 
                                               route_scratch(ws, L), st));
 }
 
+// psa_attn, and with `hstat` the first-order mode of psa_attn_hyd
+int attn_common(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar,
+                const float* vsum, const float* hstat, const int* row_ptr, const int* col_idx, size_t col_capacity,
+                const float* row_max, int B, int H, int N, int d, int block_size, int causal, psa_bf16_t* out,
+                float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !kbar || !vsum || !row_ptr || !col_idx || !out || !workspace) return PSA_ERR_ARG;
+  int s = check_shape(B, H, N, d, block_size);
+  if (s != PSA_OK) return s;
+  if (causal != 0 && causal != 1) return PSA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kbar) ||
+      !aligned16(vsum) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (reinterpret_cast<uintptr_t>(row_max) & 3u) ||
+      (reinterpret_cast<uintptr_t>(hstat) & 15u))
+    return PSA_ERR_ARG;
+  const long long bh = static_cast<long long>(B) * H;
+  const int M = N / kBlock;
+  const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
+  if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
+  if ((s = check_device({q, out, workspace})) != PSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
+  if (e != cudaSuccess) return PSA_ERR_CUDA;
+  uint16_t* kb16 = reinterpret_cast<uint16_t*>(ws + L.kbar_bf16);
+  uint16_t* vb16 = reinterpret_cast<uint16_t*>(ws + L.vsum_bf16);
+  e = psa::launch_stats_to_bf16(kbar, vsum, bh * M * d, kb16, vb16, st);
+  if (e != cudaSuccess) return PSA_ERR_CUDA;
+  psa::AttnLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.kbar_bf16 = kb16;
+  a.vsum_bf16 = vb16;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.col_cap = col_capacity > static_cast<size_t>(LLONG_MAX) ? LLONG_MAX : static_cast<long long>(col_capacity);
+  a.row_max = row_max;
+  a.stall = psa::take_stall_request();
+  a.out = out;
+  a.lse = lse;
+  a.BH = static_cast<int>(bh);
+  a.N = N;
+  a.M = M;
+  a.d = d;
+  a.causal = causal;
+  a.dense = 0;
+  a.status = reinterpret_cast<int*>(ws);
+  a.fixup_count = reinterpret_cast<int*>(ws) + 1;
+  a.fixup_list = reinterpret_cast<int*>(ws + L.fixup_list);
+  a.fixup_count2 = reinterpret_cast<int*>(ws) + 2;
+  a.sched = reinterpret_cast<int*>(ws) + 3;
+  a.fixup_list2 = reinterpret_cast<int*>(ws + L.fixup_list2);
+  a.row_lse2 = reinterpret_cast<float*>(ws + L.row_lse2);
+  a.hyd = hstat != nullptr;
+  a.hyd_w = hstat ? reinterpret_cast<float*>(ws + L.hyd_w) : nullptr;
+  if ((e = psa::launch_attn(a, st)) != cudaSuccess) return PSA_ERR_CUDA;
+  if (hstat)
+    e = psa::launch_hyd_apply(q, hstat, a.hyd_w, out, a.BH, N, d, a.status, st);
+  return cuda_status(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -271,52 +340,38 @@ int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, cons
              const int* row_ptr, const int* col_idx, size_t col_capacity, const float* row_max, int B, int H,
              int N, int d, int block_size, int causal, psa_bf16_t* out, float* lse, void* workspace,
              size_t workspace_bytes, void* stream) {
-  if (!q || !k || !v || !kbar || !vsum || !row_ptr || !col_idx || !out || !workspace) return PSA_ERR_ARG;
-  int s = check_shape(B, H, N, d, block_size);
+  return attn_common(q, k, v, kbar, vsum, nullptr, row_ptr, col_idx, col_capacity, row_max, B, H, N, d, block_size,
+                     causal, out, lse, workspace, workspace_bytes, stream);
+}
+
+int psa_attn_hyd(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar,
+                 const float* vsum, const float* hstat, const int* row_ptr, const int* col_idx, size_t col_capacity,
+                 const float* row_max, int B, int H, int N, int d, int block_size, int causal, psa_bf16_t* out,
+                 float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!hstat) return PSA_ERR_ARG;
+  return attn_common(q, k, v, kbar, vsum, hstat, row_ptr, col_idx, col_capacity, row_max, B, H, N, d, block_size,
+                     causal, out, lse, workspace, workspace_bytes, stream);
+}
+
+int psa_hyd_stat(const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar, const float* vsum, int B, int H,
+                 int N, int d, float* hstat, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!k || !v || !kbar || !vsum || !hstat || !workspace) return PSA_ERR_ARG;
+  int s = check_shape(B, H, N, d, kBlock);
   if (s != PSA_OK) return s;
-  if (causal != 0 && causal != 1) return PSA_ERR_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kbar) ||
-      !aligned16(vsum) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (reinterpret_cast<uintptr_t>(row_max) & 3u))
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kbar) || !aligned16(vsum) || !aligned16(hstat) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return PSA_ERR_ARG;
   const long long bh = static_cast<long long>(B) * H;
   const int M = N / kBlock;
   const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
   if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
-  if ((s = check_device({q, out, workspace})) != PSA_OK) return s;
+  if ((s = check_device({k, hstat, workspace})) != PSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
-  if (e != cudaSuccess) return PSA_ERR_CUDA;
-  uint16_t* kb16 = reinterpret_cast<uint16_t*>(ws + L.kbar_bf16);
-  uint16_t* vb16 = reinterpret_cast<uint16_t*>(ws + L.vsum_bf16);
-  e = psa::launch_stats_to_bf16(kbar, vsum, bh * M * d, kb16, vb16, st);
-  if (e != cudaSuccess) return PSA_ERR_CUDA;
-  psa::AttnLaunch a;
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  a.kbar_bf16 = kb16;
-  a.vsum_bf16 = vb16;
-  a.kbar32 = kbar;
-  a.vsum32 = vsum;
-  a.row_ptr = row_ptr;
-  a.col_idx = col_idx;
-  a.col_cap = col_capacity > static_cast<size_t>(LLONG_MAX) ? LLONG_MAX : static_cast<long long>(col_capacity);
-  a.row_max = row_max;
-  a.stall = psa::take_stall_request();
-  a.out = out;
-  a.lse = lse;
-  a.BH = static_cast<int>(bh);
-  a.N = N;
-  a.M = M;
-  a.d = d;
-  a.causal = causal;
-  a.dense = 0;
-  a.status = reinterpret_cast<int*>(ws);
-  a.fixup_count = reinterpret_cast<int*>(ws) + 1;
-  a.fixup_list = reinterpret_cast<int*>(ws + L.fixup_list);
-  return cuda_status(psa::launch_attn(a, st));
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
+  return cuda_status(psa::launch_hyd_stat(k, v, kbar, vsum, static_cast<int>(bh), N, d,
+                                          reinterpret_cast<float*>(ws + L.hyd_partial), hstat,
+                                          reinterpret_cast<int*>(ws), st));
 }
 
 int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int B, int H, int N, int d,
@@ -358,6 +413,10 @@ int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int
   a.status = reinterpret_cast<int*>(ws);
   a.fixup_count = reinterpret_cast<int*>(ws) + 1;
   a.fixup_list = reinterpret_cast<int*>(ws + L.fixup_list);
+  a.fixup_count2 = reinterpret_cast<int*>(ws) + 2;
+  a.sched = reinterpret_cast<int*>(ws) + 3;
+  a.fixup_list2 = reinterpret_cast<int*>(ws + L.fixup_list2);
+  a.row_lse2 = reinterpret_cast<float*>(ws + L.row_lse2);
   return cuda_status(psa::launch_attn(a, st));
 }
 
@@ -367,14 +426,15 @@ int psa_test_stall_next_attn(int on) {
   return PSA_OK;
 }
 
-int psa_read_fixup_count(const void* workspace, int* count, void* stream) {
-  if (!workspace || !count) return PSA_ERR_ARG;
+int psa_read_fixup_count(const void* workspace, int* rerun, int* exact, void* stream) {
+  if (!workspace || !rerun || !exact) return PSA_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return PSA_ERR_CUDA;
-  int v = 0;
-  if (cudaMemcpy(&v, static_cast<const int*>(workspace) + 1, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+  int v[2] = {0, 0};
+  if (cudaMemcpy(v, static_cast<const int*>(workspace) + 1, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
     return PSA_ERR_CUDA;
-  *count = v;
+  *rerun = v[0];
+  *exact = v[1];
   return PSA_OK;
 }
 

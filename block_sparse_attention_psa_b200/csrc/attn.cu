@@ -74,15 +74,26 @@ struct Cfg {
   static constexpr int kMiscBytes = 256 + 256 + (8 * 128 + 8) * 4 + 128 * 4 + 64 * 4 + kMaxBlocks / 8 +
                                     kColCache * 4;
   static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+  // first-order (hyd) mode: an all-ones bf16 operand (128 rows x 16, no
+  // swizzle: 4 KB) whose product with P^T gives each query's column sum of
+  // the 0th-order weights, and the two warpgroups' copies of those sums
+  static constexpr int kOffOnes = kOffMisc + kMiscBytes;
+  static constexpr int kOffRt = kOffOnes + 4096;
+  static constexpr int kSmemBytesHyd = kOffRt + 2 * 64 * 4 + 1024;
+  static_assert(kOffOnes % 16 == 0, "no-swizzle operand alignment");
+  static_assert(kSmemBytesHyd <= 232448, "shared memory of one CTA");
   // kind::f16, bf16 x bf16 -> f32.  GEMM1: M=128 keys, N=64 queries, both
   // K-major.  GEMM2: M=128 (feature rows), N=64 queries, both MN-major.
   static constexpr uint32_t kIdesc1 = idesc_bf16_f32(128, 64, 0, 0);
   static constexpr uint32_t kIdesc2 = idesc_bf16_f32(128, 64, 1, 1);
+  // hyd mode: R[128 x 64 queries] += ONES[128 x 128 keys] . P^T (A K-major)
+  static constexpr uint32_t kIdescOnes = idesc_bf16_f32(128, 64, 0, 1);
 };
 
 struct Params {
   const uint16_t* q;          // bf16 [BH, N, D]: block means for the stabiliser
   const uint16_t* kbar16;     // bf16 [BH, M, D]: pooled keys
+  const uint16_t* vsum16;     // bf16 [BH, M, D]: pooled value sums (the 0th-order operands)
   const int* row_ptr;
   const int* col_idx;
   long long col_cap;
@@ -93,8 +104,15 @@ struct Params {
   int stall;         // test hook: CTA 0 withholds its first S^T hand-off
   float scale_log2;  // log2(e) / sqrt(d)
   int* status;
-  int* fixup_count;
-  int* fixup_list;
+  int* fixup_count;   // units whose denominator left the safe range: count ...
+  int* fixup_list;    // ... and their unit ids
+  float* hyd_w;      // hyd mode: per query, the 0th-order share of its softmax [BH * N]
+  float* lse2_out;   // first pass: per query, log2 of its denominator incl. the stabiliser [BH * N]
+  // rerun (FIX) mode: the units to recompute (the first pass's list) and each
+  // query's log2 denominator from the first pass, used as its own stabiliser
+  const int* fix_src_count;
+  const int* fix_src_list;
+  const float* row_lse2;
 };
 
 // Everything every role needs to agree on about one work unit.
@@ -213,14 +231,20 @@ __device__ __forceinline__ void reg_alloc() {
 // `keep`); 2: diagonal block under the causal mask (key kj visible to query
 // q iff kj <= q).
 // The scale/bias and the denominator sums use packed fp32 pair instructions.
-template <int kMode, int kHalf>
-__device__ __forceinline__ void exp_half(const float (&sv)[64], float bias, float (&lsum)[64], float sl, int kj,
-                                         bool keep, uint32_t (&pk)[16]) {
+// kPerQ: the stabiliser is per query column (rerun mode), read from `fb`.
+template <int kMode, int kHalf, bool kPerQ>
+__device__ __forceinline__ void exp_half(const float (&sv)[64], float bias, const float* fb, float (&lsum)[64],
+                                         float sl, int kj, bool keep, uint32_t (&pk)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int q0 = 32 * kHalf + 2 * i, q1 = q0 + 1;
     float x0, x1;
-    ffma2(x0, x1, sv[q0], sv[q1], sl, sl, bias, bias);
+    if (kPerQ) {
+      const float2 bb = *reinterpret_cast<const float2*>(fb + q0);
+      ffma2(x0, x1, sv[q0], sv[q1], sl, sl, bb.x, bb.y);
+    } else {
+      ffma2(x0, x1, sv[q0], sv[q1], sl, sl, bias, bias);
+    }
     float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
     if (kMode == 1) {
       e0 = keep ? e0 : 0.f;
@@ -237,7 +261,7 @@ __device__ __forceinline__ void exp_half(const float (&sv)[64], float bias, floa
   }
 }
 
-template <int D>
+template <int D, bool HYD, bool FIX>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
@@ -273,8 +297,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* invl = qbs + 128;
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(invl + 64);
   int* cols = reinterpret_cast<int*>(bitmap + kMaxBlocks / 32);
+  constexpr uint32_t kTmemCols = HYD ? 512 : 256;  // hyd: + two R buffers [64 cols] at column 256
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // the units of this launch: every (head, query block), or in rerun mode the
+  // first pass's list (unit ids from it)
+  const int units = FIX ? *p.fix_src_count : p.units;
+  auto uid = [&](int u) { return FIX ? __ldg(p.fix_src_list + u) : u; };
+  if constexpr (HYD) {
+    // all-ones operand (bf16 1.0 = 0x3f80), read by the tensor core through the async proxy
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::kOffOnes);
+    for (int i = threadIdx.x; i < 1024; i += kThreads) ones[i] = 0x3f803f80u;
+    fence_async_shared();
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -302,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmVb);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -323,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int qc = 0;
     bool ok = true;
     int ul = 0;
-    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ul) {
-      const Unit x = make_unit(u, p);
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+      const Unit x = make_unit(uid(u), p);
       const int qb = ul & 1;
       if (keys && lane == 0) {
         ok = mbar_wait(&q_empty[qb], ((ul >> 1) & 1) ^ 1, abort_flag, p.status);
@@ -405,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int sc = 0;
       bool ok = true;
       int ul = 0;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ul) {
-        const Unit x = make_unit(u, p);
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+        const Unit x = make_unit(uid(u), p);
         const int qb = ul & 1;
         if (!(ok = mbar_wait(&q_full[qb], (ul >> 1) & 1, abort_flag, p.status))) break;
         const uint64_t dq = dQ0 + qb * kQStep;
@@ -441,13 +476,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // V viewed MN-major: feature atoms 16 KB apart (d = 64: the second
       // atom repeats the first and its output rows are never read)
       const uint64_t dP0 = sdesc_sw128(smem_u32(sP), 16, 1024);
+      // all-ones A operand (hyd mode): 16 core matrices of 8 rows along M
+      // (256 B apart), 2 along K (128 B apart) -- 4 KB, every byte 1.0
+      const uint64_t dOnes = sdesc_noswizzle(smem_u32(smem + C::kOffOnes), 128, 256);
+      (void)dOnes;
       constexpr uint64_t kKVStep = C::kKVBytes >> 4, kPStep = C::kPBytes >> 4;
       int sc = 0;
       int used[2] = {0, 0};  // GEMM2s issued on each buffer parity
       bool ok = true;
       int ul = 0;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++ul) {
-        const Unit x = make_unit(u, p);
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+        const Unit x = make_unit(uid(u), p);
         const int ob = ul & 1;
         const int g2_total = x.n_a2 + x.n_e;
         for (int g = 0; g < g2_total; ++g, ++sc) {
@@ -462,6 +501,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_mma_bf16(dt, a, b, C::kIdesc2, g == 0 ? 0u : 1u);
 #pragma unroll
           for (int kk = 1; kk < 8; ++kk) tc_mma_bf16(dt, a + 128 * kk, b + 128 * kk, C::kIdesc2, 1u);
+          if constexpr (HYD) {
+            if (g < x.n_a2) {
+              // pooled tile: R[unit parity] += ONES . P^T, the column sums of this
+              // tile's 0th-order weights (every row of R holds the same sums)
+              const uint32_t rt = tbase + 256 + 64 * ob;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                tc_mma_bf16(rt, dOnes, b + 128 * kk, C::kIdescOnes, (g == 0 && kk == 0) ? 0u : 1u);
+            }
+          }
           tc_commit(&g2_done[pb]);
           if (g == g2_total - 1) tc_commit(&o_full[ob]);
           if (pb) ++used[1]; else ++used[0];
@@ -504,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // unit's row_ptr pair and rmax its router row maximum, loaded by the
     // caller ahead of time.
     auto prologue = [&](int u, int a, int b, float rmax) {
-        x = make_unit_with(u, p, a, b);
+        x = make_unit_with(uid(u), p, a, b);
         if (!p.dense) {
           // mark the listed blocks (A2 skips them), cache the list, validate it
           bool bad = x.bad;
@@ -523,6 +572,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
   #pragma unroll
         for (int q = 0; q < 64; ++q) lsum[q] = 0.f;
+        if constexpr (FIX) {
+          // rerun: each query's own log2 denominator from the first pass is its
+          // stabiliser (qbs[q] = -that), so its sum lands near 1; a query whose
+          // first-pass sum was not finite gets 0 and is flagged again
+          if (gtid < 64) {
+            const float l2 = p.row_lse2[static_cast<size_t>(x.row) * 64 + gtid];
+            qbs[gtid] = isfinite(l2) ? -l2 : 0.f;
+          }
+          named_barrier_sync(1, 256);
+          c2 = 0.f;
+          bias = 0.f;
+          return;
+        }
         // Stabiliser of the whole query block (log2 units): c2 = max over the
         // candidate blocks of qbar_I . kbar_J / sqrt(d) * log2(e) + log2(64),
         // with qbar_I the mean of the block's queries.  Any constant within a
@@ -596,8 +658,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int na = 0, nb = 0;
     float nrmax = 0.f;
     auto load_next = [&](int un) {
-      if (un >= p.units) return;
-      const int row = unit_row(un, p);
+      if (un >= units) return;
+      const int row = unit_row(uid(un), p);
       if (!p.dense) {
         na = __ldg(p.row_ptr + row);
         nb = __ldg(p.row_ptr + row + 1);
@@ -605,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.row_max) nrmax = __ldg(p.row_max + row);
     };
     const int nw_all = (p.M + 31) / 32;  // bitmap words of the widest candidate range
-    bool go = static_cast<int>(blockIdx.x) < p.units;
+    bool go = static_cast<int>(blockIdx.x) < units;
     if (go) {
       load_next(blockIdx.x);
       if (gtid == 0) *stop_s = *abort_flag;
@@ -650,14 +712,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kj = trow & 63;
         uint32_t pk[32];
         if (mode == 0) {
-          exp_half<0, 0>(sv, bias, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-          exp_half<0, 1>(sv, bias, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+          exp_half<0, 0, FIX>(sv, bias, qbs, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+          exp_half<0, 1, FIX>(sv, bias, qbs, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
         } else if (mode == 1) {
-          exp_half<1, 0>(sv, bias, lsum, p.scale_log2, kj, valid, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-          exp_half<1, 1>(sv, bias, lsum, p.scale_log2, kj, valid, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+          exp_half<1, 0, FIX>(sv, bias, qbs, lsum, p.scale_log2, kj, valid, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+          exp_half<1, 1, FIX>(sv, bias, qbs, lsum, p.scale_log2, kj, valid, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
         } else if (mode == 2) {
-          exp_half<2, 0>(sv, bias, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-          exp_half<2, 1>(sv, bias, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+          exp_half<2, 0, FIX>(sv, bias, qbs, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+          exp_half<2, 1, FIX>(sv, bias, qbs, lsum, p.scale_log2, kj, true, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) pk[i] = 0u;
@@ -682,15 +744,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool good = l >= 0x1p-60f && l <= 0x1p60f;  // false for NaN
         invl[gtid] = good ? 1.0f / l : 0.f;
         if (!good) *unit_flag = 1;
-        if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + gtid] = (c2 + __log2f(l)) * kLn2;
+        const float lse2 = (FIX ? -qbs[gtid] : c2) + __log2f(l);
+        if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + gtid] = lse2 * kLn2;
+        if (!FIX) p.lse2_out[static_cast<size_t>(x.row) * 64 + gtid] = lse2;
       }
-      const bool more = u + static_cast<int>(gridDim.x) < p.units;
+      const bool more = u + static_cast<int>(gridDim.x) < units;
       if (gtid == 0) *stop_s = *abort_flag;
       if ((gtid & 127) == 0) bulk_wait_read0();  // the last unit's store has read the staging tile
       if (more && !p.dense)
         for (int i = gtid; i < nw_all; i += 256) bitmap[i] = 0u;
       named_barrier_sync(1, 256);
       const int row_done = x.row;
+      const bool had_a2 = x.n_a2 > 0;
       // the next unit's setup overlaps the wait for this unit's last GEMM2
       go = more && !*stop_s;
       if (go) {
@@ -715,17 +780,43 @@ __global__ void __launch_bounds__(kThreads, 1)
               st[(32 * h + q) * D + trow] = __float2bfloat16_rn(ov[q] * invl[32 * h + q]);
           }
         }
+        if constexpr (HYD) {
+          // the first warp of the storing warpgroup (TMEM lanes 0..31) reads the
+          // 64 column sums of this unit's 0th-order weights before the buffer is freed
+          float* rts = reinterpret_cast<float*>(smem + C::kOffRt) + 64 * w;
+          if (wq == 0 && had_a2) {
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+              float rv[32];
+              tmem_ld32(tbase + 256 + 64 * ob + 32 * h, rv);
+              tc_wait_ld();
+              if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                  *reinterpret_cast<float4*>(rts + 32 * h + i) = make_float4(rv[i], rv[i + 1], rv[i + 2], rv[i + 3]);
+              }
+            }
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&o_empty[ob]);
         fence_async_shared();
         named_barrier_sync(2 + w, 128);
+        if constexpr (HYD) {
+          // w_q = (sum of the 0th-order weights) / denominator, per query
+          const int qq = gtid & 127;
+          if (qq < 64) {
+            const float* rts = reinterpret_cast<const float*>(smem + C::kOffRt) + 64 * w;
+            p.hyd_w[static_cast<size_t>(row_done) * 64 + qq] = had_a2 ? rts[qq] * invl[qq] : 0.f;
+          }
+        }
         if ((gtid & 127) == 0) {
           bulk_store(p.out + static_cast<size_t>(row_done) * 64 * D, sOut, C::kOutBytes);
           bulk_commit();
           if (*unit_flag) {
             const int slot = atomicAdd(p.fixup_count, 1);
-            p.fixup_list[slot] = u;
+            p.fixup_list[slot] = uid(u);
             *unit_flag = 0;
           }
         }
@@ -738,20 +829,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, 256);
+    tmem_dealloc(tbase, kTmemCols);
   }
 }
 
 // ------------------------------------------------------------------ fixup
 // Exact two-pass recomputation (fp32, CUDA cores) of the units whose
-// denominator left the safe range under the fixed stabiliser.  One CTA of
-// 64 threads per listed unit, one thread per query row.  Rare path.
+// denominator left the safe range under the fixed stabiliser: the same terms
+// as the tensor-core sweep (the 0th-order ones with the same bf16 pooled
+// keys and value sums), with each query's own maximum as its stabiliser.
+// One CTA of 64 threads per listed unit, one thread per query row.
 template <int D>
 __global__ void __launch_bounds__(64) fixup_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k,
-                                                   const __nv_bfloat16* __restrict__ v,
-                                                   const float* __restrict__ kbar, const float* __restrict__ vsum,
-                                                   Params p, int N) {
+                                                   const __nv_bfloat16* __restrict__ v, Params p, int N) {
   extern __shared__ float fx_sm[];
   float(*qs)[D + 1] = reinterpret_cast<float(*)[D + 1]>(fx_sm);
   float(*num)[D + 1] = reinterpret_cast<float(*)[D + 1]>(fx_sm + 64 * (D + 1));
@@ -782,6 +873,7 @@ __global__ void __launch_bounds__(64) fixup_kernel(const __nv_bfloat16* __restri
     float m = -INFINITY;
     for (int pass = 0; pass < 2; ++pass) {
       float den = 0.f;
+      float zeroth = 0.f;  // sum of the 0th-order weights (hyd mode)
       for (int J = 0; J < x.cand; ++J) {
         const bool on = (listed[J >> 5] >> (J & 31)) & 1u;
         if (on) {
@@ -798,17 +890,20 @@ __global__ void __launch_bounds__(64) fixup_kernel(const __nv_bfloat16* __restri
               for (int c = 0; c < D; ++c) num[i][c] = fmaf(w, __bfloat162float(v[(head + j) * D + c]), num[i][c]);
             }
           }
-        } else if (J < x.pcand && kbar != nullptr) {
+        } else if (J < x.pcand) {
           const size_t kb = (static_cast<size_t>(x.bh) * p.M + J) * D;
+          const __nv_bfloat16* kb16 = reinterpret_cast<const __nv_bfloat16*>(p.kbar16);
+          const __nv_bfloat16* vs16 = reinterpret_cast<const __nv_bfloat16*>(p.vsum16);
           float a = 0.f;
-          for (int c = 0; c < D; ++c) a = fmaf(qs[i][c], kbar[kb + c], a);
+          for (int c = 0; c < D; ++c) a = fmaf(qs[i][c], __bfloat162float(kb16[kb + c]), a);
           a *= tau;
           if (pass == 0) {
             m = fmaxf(m, a + 4.1588830833596715f);  // + ln 64
           } else {
             const float w = __expf(a - m);
             den += 64.f * w;
-            for (int c = 0; c < D; ++c) num[i][c] = fmaf(w, vsum[kb + c], num[i][c]);
+            zeroth += w;
+            for (int c = 0; c < D; ++c) num[i][c] = fmaf(w, __bfloat162float(vs16[kb + c]), num[i][c]);
           }
         }
       }
@@ -816,14 +911,38 @@ __global__ void __launch_bounds__(64) fixup_kernel(const __nv_bfloat16* __restri
         const float r = 1.0f / den;
         for (int c = 0; c < D; ++c) p.out[(head + qi) * D + c] = __float2bfloat16_rn(num[i][c] * r);
         if (p.lse) p.lse[head + qi] = m + __logf(den);
+        if (p.hyd_w) p.hyd_w[head + qi] = zeroth * r;
       }
     }
   }
 }
 
-template <int D>
+// The attention kernel's shared-memory limit and register check for one
+// instantiation.
+template <int D, bool HYD, bool FIX>
+cudaError_t prepare_attn_kernel(int smem) {
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, HYD, FIX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  // The warpgroups re-split the registers the block was launched with
+  // (setmaxnreg); if the compiled kernel launched with fewer, the increase
+  // could never be satisfied.  Refuse to launch rather than wait forever.
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, attn_kernel<D, HYD, FIX>)) != cudaSuccess) return e;
+  if (fa.numRegs < kRegsLaunch || 128 * kRegsProducer + 256 * kRegsSoftmax > kThreads * fa.numRegs)
+    return cudaErrorInvalidConfiguration;
+  return cudaSuccess;
+}
+
+// Three launches: the attention sweep over every unit (fixed per-block
+// stabiliser); a rerun of the units it flagged, each query with its own
+// stabiliser from the first pass's denominator (the same tensor-core
+// kernel; its grid finds the count on the device and exits when it is 0);
+// and the exact CUDA-core recomputation of any unit the rerun still flags
+// (a first-pass sum that was not finite).
+template <int D, bool HYD>
 cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   using C = Cfg<D>;
+  constexpr int kSmem = HYD ? C::kSmemBytesHyd : C::kSmemBytes;
   CUtensorMap mq, mk, mv, mkb, mvb;
   const uint64_t bh = static_cast<uint64_t>(a.BH);
   if (encode_tensor_map_3d_bf16(&mq, a.q, D, a.N, bh, 64, 64) != CUDA_SUCCESS ||
@@ -836,6 +955,7 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   Params p;
   p.q = a.q;
   p.kbar16 = a.kbar_bf16;
+  p.vsum16 = a.vsum_bf16;
   p.row_ptr = a.row_ptr;
   p.col_idx = a.col_idx;
   p.col_cap = a.col_cap;
@@ -852,36 +972,48 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   p.fixup_count = a.fixup_count;
   p.fixup_list = a.fixup_list;
   p.stall = a.stall;
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  // The warpgroups re-split the registers the block was launched with
-  // (setmaxnreg); if the compiled kernel launched with fewer, the increase
-  // could never be satisfied.  Refuse to launch rather than wait forever.
-  cudaFuncAttributes fa;
-  if ((e = cudaFuncGetAttributes(&fa, attn_kernel<D>)) != cudaSuccess) return e;
-  if (fa.numRegs < kRegsLaunch ||
-      128 * kRegsProducer + 256 * kRegsSoftmax > kThreads * fa.numRegs)
-    return cudaErrorInvalidConfiguration;
+  p.hyd_w = HYD ? a.hyd_w : nullptr;
+  p.lse2_out = a.row_lse2;
+  p.fix_src_count = nullptr;
+  p.fix_src_list = nullptr;
+  p.row_lse2 = nullptr;
+  cudaError_t e;
+  if ((e = prepare_attn_kernel<D, HYD, false>(kSmem)) != cudaSuccess) return e;
+  if ((e = prepare_attn_kernel<D, HYD, true>(kSmem)) != cudaSuccess) return e;
   const int sms = device_sm_count();
   const int grid = p.units < sms ? p.units : sms;
-  attn_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mkb, mvb, p);
+  attn_kernel<D, HYD, false><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, mkb, mvb, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // the rerun: the first pass's list in, a second list out
+  Params r = p;
+  r.stall = 0;
+  r.fix_src_count = a.fixup_count;
+  r.fix_src_list = a.fixup_list;
+  r.row_lse2 = a.row_lse2;
+  r.lse2_out = nullptr;
+  r.fixup_count = a.fixup_count2;
+  r.fixup_list = a.fixup_list2;
+  attn_kernel<D, HYD, true><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, mkb, mvb, r);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // exact recomputation of what the rerun still flags
+  Params f = p;
+  f.fixup_count = a.fixup_count2;
+  f.fixup_list = a.fixup_list2;
   const size_t fx_smem = 128 * (D + 1) * sizeof(float) + kMaxBlocks / 8;
   if ((e = cudaFuncSetAttribute(fixup_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(fx_smem))) != cudaSuccess)
     return e;
   fixup_kernel<D><<<64, 64, fx_smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(a.q),
                                            reinterpret_cast<const __nv_bfloat16*>(a.k),
-                                           reinterpret_cast<const __nv_bfloat16*>(a.v), a.kbar32, a.vsum32, p,
-                                           a.N);
+                                           reinterpret_cast<const __nv_bfloat16*>(a.v), f, a.N);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t st) {
-  return a.d == 128 ? launch_d<128>(a, st) : launch_d<64>(a, st);
+  if (a.hyd && !a.dense) return a.d == 128 ? launch_d<128, true>(a, st) : launch_d<64, true>(a, st);
+  return a.d == 128 ? launch_d<128, false>(a, st) : launch_d<64, false>(a, st);
 }
 
 }  // namespace psa

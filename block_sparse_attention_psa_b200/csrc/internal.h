@@ -16,14 +16,18 @@ constexpr int kMaxBlocks = 16384; // M limit (bitmaps and score rows on chip)
 // Workspace layout (byte offsets, each 256-aligned).  The header holds the
 // status word and the fixup counter.
 struct WorkspaceLayout {
-  size_t header = 0;        // int status; int fixup_count; ... (256 B)
-  size_t fixup_list = 0;    // int [B*H*M]
+  size_t header = 0;        // int status, fixup_count, fixup_count2, sched[2]; ... (256 B, zeroed per call)
+  size_t fixup_list = 0;    // int [B*H*M]   units flagged by the attention sweep
+  size_t fixup_list2 = 0;   // int [B*H*M]   units still flagged by the rerun
+  size_t row_lse2 = 0;      // fp32 [B*H*N] per query log2 denominator of the sweep
   size_t kbar_bf16 = 0;     // bf16 [B*H*M*d]
   size_t vsum_bf16 = 0;     // bf16 [B*H*M*d] (value sums)
   size_t row_count = 0;     // int [B*H*M]     (threshold routing)
   size_t row_bits = 0;      // uint32 [B*H*M*ceil(M/32)]
   size_t q_split = 0;       // bf16 [3][B*H*M*d] (three-part split of qbar, routing)
   size_t k_split = 0;       // bf16 [3][B*H*M*d] (same for kbar)
+  size_t hyd_w = 0;         // fp32 [B*H*N] (first-order mode: 0th-order share per query)
+  size_t hyd_partial = 0;   // fp32 partial statistics of the first-order mode
   size_t scores = 0;        // fp32 [score_heads][M][Mp] block scores of one batch of heads
   int score_heads = 0;      // heads per routing batch
   size_t total = 0;
@@ -77,8 +81,6 @@ struct AttnLaunch {
   const uint16_t* v;
   const uint16_t* kbar_bf16;
   const uint16_t* vsum_bf16;
-  const float* kbar32;  // may be null in dense mode
-  const float* vsum32;  // may be null in dense mode
   const int* row_ptr;   // null in dense mode
   const int* col_idx;   // null in dense mode
   long long col_cap;
@@ -87,11 +89,27 @@ struct AttnLaunch {
   float* lse;
   int BH, N, M, d, causal, dense;
   int* status;
-  int* fixup_count;
+  int* fixup_count;   // units the first pass flagged (rerun with per-query stabilisers)
   int* fixup_list;
+  int* fixup_count2;  // units the rerun still flagged (exact CUDA-core path)
+  int* fixup_list2;
+  float* row_lse2;    // [BH * N]: per query, the first pass's log2 denominator
+  int* sched;         // [2] zeroed ticket counters of the attention sweep and of its rerun
   int stall;  // failure-path test hook (0 in normal use)
+  int hyd = 0;             // first-order mode: also write hyd_w (per query, 0th-order share)
+  float* hyd_w = nullptr;  // [BH * N] fp32 (hyd mode only)
 };
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t st);
+
+// hyd.cu: the first-order correction
+// partial matrices of the statistic kernel (bytes, for the workspace)
+size_t hyd_partial_bytes(int BH, int M, int d);
+// hstat[BH][d][d] = mean over the blocks J of sum_{j in J} (k_j - kbar_J) v_j^T
+cudaError_t launch_hyd_stat(const uint16_t* k, const uint16_t* v, const float* kbar, const float* vsum, int BH,
+                            int N, int d, float* partial, float* hstat, int* status, cudaStream_t st);
+// out[i] += w[i] * (q_i^T H) / sqrt(d), in place
+cudaError_t launch_hyd_apply(const uint16_t* q, const float* hstat, const float* w, uint16_t* out, int BH, int N,
+                             int d, int* status, cudaStream_t st);
 
 // api.cu: one-shot flag set by psa_test_stall_next_attn, taken by the next psa_attn
 int take_stall_request();

@@ -6,8 +6,9 @@
 // memory all comes from the framework's own pool, or real-time and
 // safety-critical loops that forbid allocation after start-up.  This entry point needs nothing from them but
 // the inputs and outputs: its scratch (the bf16 copies of the pooled keys
-// and value sums, the status word and the fixup list) lives in one
-// file-scope device array below.
+// and value sums, the status word, the fixup lists and the per-query
+// denominators the fixup rerun starts from) lives in one file-scope device
+// array below.
 //
 // That array is shared by every call on a device and keeps the previous
 // call's contents; the parts that must start at zero (status word, fixup
@@ -36,10 +37,12 @@ unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Scratch bytes the attention step needs: header, fixup list, bf16 pooled keys
-// and bf16 value sums (the same layout as the front of the workspace).
+// Scratch bytes the attention step needs: header, the first fixup list, bf16
+// pooled keys and bf16 value sums, the second fixup list and the per-query
+// log2 denominators of the first pass.
 size_t scratch_bytes(long long BH, long long M, long long d) {
-  return 256 + align256(static_cast<size_t>(BH * M) * 4) + 2 * align256(static_cast<size_t>(BH * M * d) * 2);
+  return 256 + 2 * align256(static_cast<size_t>(BH * M) * 4) + 2 * align256(static_cast<size_t>(BH * M * d) * 2) +
+         align256(static_cast<size_t>(BH * M * 64) * 4);
 }
 
 typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
@@ -122,6 +125,8 @@ int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
   const size_t off_fix = 256;
   const size_t off_kb = off_fix + align256(static_cast<size_t>(bh * M) * 4);
   const size_t off_vs = off_kb + align256(static_cast<size_t>(bh * M * d) * 2);
+  const size_t off_fix2 = off_vs + align256(static_cast<size_t>(bh * M * d) * 2);
+  const size_t off_lse2 = off_fix2 + align256(static_cast<size_t>(bh * M) * 4);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the status word and the fixup counter must start at zero on every call
   if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
@@ -134,8 +139,6 @@ int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
   a.v = v;
   a.kbar_bf16 = kb16;
   a.vsum_bf16 = vs16;
-  a.kbar32 = kbar;
-  a.vsum32 = vsum;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
   a.col_cap = col_capacity > static_cast<size_t>(LLONG_MAX) ? LLONG_MAX : static_cast<long long>(col_capacity);
@@ -152,6 +155,10 @@ int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
   a.status = reinterpret_cast<int*>(ws);
   a.fixup_count = reinterpret_cast<int*>(ws) + 1;
   a.fixup_list = reinterpret_cast<int*>(ws + off_fix);
+  a.fixup_count2 = reinterpret_cast<int*>(ws) + 2;
+  a.sched = reinterpret_cast<int*>(ws) + 3;
+  a.fixup_list2 = reinterpret_cast<int*>(ws + off_fix2);
+  a.row_lse2 = reinterpret_cast<float*>(ws + off_lse2);
   if (psa::launch_attn(a, st) != cudaSuccess) return PSA_ERR_CUDA;
   if (status && cudaMemcpyAsync(status, ws, sizeof(int), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return PSA_ERR_CUDA;

@@ -111,6 +111,14 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, void* smem_d
       : "memory");
 }
 
+// 3-D tiled store shared -> global (bulk group): the box at element
+// coordinates (x, y, z); rows outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 // Bulk (non-tensor) copy shared -> global; both addresses 16-byte aligned,
 // size a multiple of 16.
 __device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
@@ -192,6 +200,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
   d |= 1ull << 46;   // descriptor version for sm_100
   d |= 2ull << 61;   // SWIZZLE_128B
+  return d;
+}
+
+// Shared-memory matrix descriptor without swizzle (K-major core matrices of
+// 8 rows x 16 bytes): lbo = byte distance between core matrices along K,
+// sbo = along M/N.
+__device__ __forceinline__ uint64_t sdesc_noswizzle(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= 1ull << 46;   // descriptor version for sm_100; layout bits [61, 64) = 0: no swizzle
   return d;
 }
 

@@ -32,7 +32,7 @@ PSA_ERR_DEVICE = 8
 EXPORTS = ("psa_status_string", "psa_version", "psa_workspace_size", "psa_route_capacity", "psa_pool",
            "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense", "psa_read_status",
            "psa_attn_noalloc", "psa_route_thresh_prob", "psa_test_stall_next_attn",
-           "psa_read_fixup_count")
+           "psa_read_fixup_count", "psa_hyd_stat", "psa_attn_hyd")
 
 _lib = None
 
@@ -57,7 +57,9 @@ def _declare(L: ctypes.CDLL) -> None:
         "psa_attn": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, Z, P]),
         "psa_dense": (I, [P, P, P, I, I, I, I, I, P, P, P, Z, P]),
         "psa_read_status": (I, [P, ctypes.POINTER(I), P]),
-        "psa_read_fixup_count": (I, [P, ctypes.POINTER(I), P]),
+        "psa_read_fixup_count": (I, [P, ctypes.POINTER(I), ctypes.POINTER(I), P]),
+        "psa_hyd_stat": (I, [P, P, P, P, I, I, I, I, P, P, Z, P]),
+        "psa_attn_hyd": (I, [P, P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, Z, P]),
         "psa_test_stall_next_attn": (I, [I]),
         "psa_attn_noalloc": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, P]),
     }
@@ -287,6 +289,47 @@ def psa_attn(q, k, v, kbar, vsum, row_ptr, col_idx, causal: bool = False, block_
     return (out, lse) if lse is not None else out
 
 
+def psa_hyd_stat(k, v, kbar, vsum, ws=None, out=None, stream=None):
+    """The first-order correction's global statistic: float32 [B, H, d, d],
+    the mean over a head's blocks of sum_j (k_j - kbar_J) v_j^T."""
+    B, H, N, d = _expect_qkv(k, v, v)
+    M = N // 64
+    _expect("kbar", kbar, k, (B, H, M, d), torch.float32)
+    _expect("vsum", vsum, k, (B, H, M, d), torch.float32)
+    if ws is None:
+        ws = workspace(B, H, N, d, k.device)
+    if out is None:
+        out = torch.empty(B, H, d, d, dtype=torch.float32, device=k.device)
+    _expect_ws(ws, k, B, H, N, d)
+    _expect("hstat", out, k, (B, H, d, d), torch.float32)
+    _call("psa_hyd_stat", k, _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), B, H, N, d, _ptr(out), _ptr(ws),
+          ws.numel(), _stream(stream, k))
+    return out
+
+
+def psa_attn_hyd(q, k, v, kbar, vsum, hstat, row_ptr, col_idx, causal: bool = False, block_size: int = 64,
+                 ws=None, out=None, lse=None, want_lse: bool = False, row_max=None, stream=None):
+    """psa_attn plus the first-order term of the unselected blocks with the
+    global statistic ``hstat`` (float32 [B, H, d, d], from psa_hyd_stat)."""
+    B, H, N, d = _expect_qkv(q, k, v)
+    M = N // block_size if block_size > 0 else 0
+    _expect_attn_inputs(q, kbar, vsum, row_ptr, col_idx, row_max, B, H, M, d)
+    _expect("hstat", hstat, q, (B, H, d, d), torch.float32)
+    if ws is None:
+        ws = workspace(B, H, N, d, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    _expect_ws(ws, q, B, H, N, d)
+    _expect("out", out, q, (B, H, N, d), torch.bfloat16)
+    _expect("lse", lse, q, (B, H, N), torch.float32)
+    _call("psa_attn_hyd", q, _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(hstat), _ptr(row_ptr),
+          _ptr(col_idx), col_idx.numel(), _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out),
+          _ptr(lse), _ptr(ws), ws.numel(), _stream(stream, q))
+    return (out, lse) if lse is not None else out
+
+
 def psa_dense(q, k, v, causal: bool = False, ws=None, out=None, lse=None, want_lse: bool = False,
               stream=None):
     """Dense softmax attention through the same tensor-core kernel."""
@@ -340,19 +383,21 @@ def psa_read_status(ws, stream=None) -> int:
     return int(st.value)
 
 
-def psa_read_fixup_count(ws, stream=None) -> int:
-    """Synchronise the stream and return how many query blocks the last
-    attention call on ``ws`` recomputed through its exact fixup path."""
+def psa_read_fixup_count(ws, stream=None):
+    """Synchronise the stream and return (rerun, exact): the query blocks the
+    last attention call on ``ws`` recomputed with per-query stabilisers on the
+    tensor cores, and those of them that needed the exact CUDA-core path."""
     _expect("ws", ws, dtype=torch.uint8, min_numel=256)
-    n = ctypes.c_int(-1)
-    _call("psa_read_fixup_count", ws, _ptr(ws), ctypes.byref(n), _stream(stream, ws))
-    return int(n.value)
+    rerun, exact = ctypes.c_int(-1), ctypes.c_int(-1)
+    _call("psa_read_fixup_count", ws, _ptr(ws), ctypes.byref(rerun), ctypes.byref(exact), _stream(stream, ws))
+    return int(rerun.value), int(exact.value)
 
 
 def psa_forward(q, k, v, mode: str = "topk", density: float = 0.15, alpha: float = 0.5,
-                causal: bool = False, keep_first: bool = False, ws=None, stream=None):
+                causal: bool = False, keep_first: bool = False, hyd: bool = False, ws=None, stream=None):
     """The whole path in one call (pool -> route -> attention), as the usage
     line of the PISA summary calls it: f(q, k, v, density=0.15, block_size=64).
+    ``hyd`` adds the first-order correction with the global statistic.
     Returns (out, (row_ptr, col_idx, nnz, row_max))."""
     B, H, N, d = _shape(q)
     if ws is None:
@@ -366,5 +411,10 @@ def psa_forward(q, k, v, mode: str = "topk", density: float = 0.15, alpha: float
         csr = psa_route_thresh_prob(qbar, kbar, alpha, causal, keep_first, ws=ws, stream=stream)
     else:
         raise ValueError("mode must be 'topk', 'thresh' or 'thresh_prob'")
-    out = psa_attn(q, k, v, kbar, vsum, csr[0], csr[1], causal, ws=ws, row_max=csr[3], stream=stream)
+    if hyd:
+        hstat = psa_hyd_stat(k, v, kbar, vsum, ws=ws, stream=stream)
+        out = psa_attn_hyd(q, k, v, kbar, vsum, hstat, csr[0], csr[1], causal, ws=ws, row_max=csr[3],
+                           stream=stream)
+    else:
+        out = psa_attn(q, k, v, kbar, vsum, csr[0], csr[1], causal, ws=ws, row_max=csr[3], stream=stream)
     return out, csr

@@ -201,6 +201,43 @@ PSA_API int psa_attn(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * f-1. The global statistic of the first-order ("hyd") correction [PISA
+ * summary, "Why approximating unselected blocks keeps softmax intact" and
+ * FAQ "Why a global first-order correction?": to first order around the
+ * block-mean key, an unselected block J adds e^{a_iJ} H_J^T q_i / sqrt(d) to
+ * the numerator, H_J = sum_{j in J} (k_j - kbar_J) v_j^T, and the pages use
+ * one global statistic in place of the per-block matrices; reading taken:
+ * the mean of H_J over the blocks of a head]:
+ *   hstat[b,h] = (1/M) sum_J sum_{j in J} (k_j - kbar_J) v_j^T
+ * float32 [B,H,d,d], row = key feature, column = value feature.
+ * Inputs: k, v bf16 [B,H,N,d]; kbar, vsum float32 [B,H,M,d] from psa_pool.
+ * `workspace` (psa_workspace_size bytes) holds the partial sums; the call
+ * resets its status word.  Errors: PSA_ERR_ARG, PSA_ERR_SHAPE,
+ * PSA_ERR_UNSUPPORTED, PSA_ERR_CAPACITY, PSA_ERR_DEVICE, PSA_ERR_CUDA.
+ */
+PSA_API int psa_hyd_stat(const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar, const float* vsum,
+                         int B, int H, int N, int d, float* hstat, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
+ * f-1. Attention with the first-order correction of the unselected blocks
+ * [same sources as psa_hyd_stat]: psa_attn's output plus, for each query,
+ *   sum_{J unlisted candidate} e^{a_iJ} (hstat^T q_i) / sqrt(d)
+ * in the numerator (the denominator is psa_attn's), i.e.
+ *   out_i = out0_i + w_i (q_i^T hstat) / sqrt(d),
+ *   w_i = sum_J e^{a_iJ} / den_i,
+ * with out0 and den the 0th-order output and denominator; lse is
+ * psa_attn's.  hstat: float32 [B,H,d,d] from psa_hyd_stat (any statistic of
+ * that shape may be passed).  Other arguments, workspace and errors as
+ * psa_attn.
+ */
+PSA_API int psa_attn_hyd(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v,
+                         const float* kbar, const float* vsum, const float* hstat,
+                         const int* row_ptr, const int* col_idx, size_t col_capacity,
+                         const float* row_max, int B, int H, int N, int d, int block_size, int causal,
+                         psa_bf16_t* out, float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Dense attention (density = 1: every candidate block exact) through the
  * same tensor-core kernel: the comparison baseline [PISA summary, "first
  * check: compare dense and PISA outputs on the same seed and input";
@@ -218,9 +255,10 @@ PSA_API int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t
  * memory (the method's sources have no counterpart: this is an interface
  * choice).  Same computation, arguments and errors as psa_attn, minus the
  * workspace: the scratch (bf16 pooled keys and value sums, status word,
- * fixup list) lives in a 16 MiB array inside the library, so shapes need
- * 256 + 4*B*H*M + 4*B*H*M*d bytes (each part rounded up to 256 bytes) to fit
- * in 16 MiB, else PSA_ERR_CAPACITY.  The first call on a device looks up the
+ * fixup lists, per-query denominators of the fixup rerun) lives in a 16 MiB
+ * array inside the library, so shapes need
+ * 256 + 8*B*H*M + 256*B*H*M + 4*B*H*M*d bytes (each part rounded up to 256
+ * bytes) to fit in 16 MiB, else PSA_ERR_CAPACITY.  The first call on a device looks up the
  * array's device address (make it before any stream capture); so does the
  * first call after a device reset, which loads the library's device code
  * anew.  Every call on a device shares the array: calls whose work overlaps
@@ -255,15 +293,19 @@ PSA_API int psa_test_stall_next_attn(int on);
 PSA_API int psa_read_status(const void* workspace, int* status, void* stream);
 
 /*
- * Synchronises `stream`, then copies into *count (host pointer) the number of
- * query blocks (64 rows each) that the last psa_attn / psa_dense call on
- * `workspace` recomputed through its exact fixup path: the blocks with a row
- * whose softmax denominator, under the kernel's fixed per-block stabiliser,
- * left [2^-60, 2^60] (an implementation detail with no counterpart in the
- * method's sources; it measures how often the slow path ran).  Returns
- * PSA_OK or PSA_ERR_CUDA.
+ * Synchronises `stream`, then reports (host pointers) how often the last
+ * psa_attn / psa_attn_hyd / psa_dense call on `workspace` left its fast path
+ * (an implementation detail with no counterpart in the method's sources):
+ *   *rerun = query blocks (64 rows each) with a row whose softmax
+ *            denominator, under the kernel's fixed per-block stabiliser,
+ *            left [2^-60, 2^60]; they were recomputed on the tensor cores
+ *            with each query's own stabiliser (from the first pass's sum);
+ *   *exact = those of them that the rerun still could not bring into range
+ *            (a first-pass sum that was not finite), recomputed by the
+ *            exact two-pass CUDA-core path.
+ * Returns PSA_OK, PSA_ERR_ARG or PSA_ERR_CUDA.
  */
-PSA_API int psa_read_fixup_count(const void* workspace, int* count, void* stream);
+PSA_API int psa_read_fixup_count(const void* workspace, int* rerun, int* exact, void* stream);
 
 #ifdef __cplusplus
 }

@@ -161,6 +161,7 @@ def test_binding_signatures_match_the_header():
 
 def test_workspace_size_holds_the_documented_parts():
     """psa_workspace_size = pooled data O(B*H*M*d) + threshold masks + the
+    first-order mode's per-query weights and partial statistics + the
     block-score matrices of as many heads as fit 256 MB (at least one head,
     4*M*Mp bytes, Mp = M rounded up to 128)."""
     def parts(B, H, M, d):
@@ -168,16 +169,24 @@ def test_workspace_size_holds_the_documented_parts():
         Mp = -(-M // 128) * 128
         head = 4 * M * Mp
         heads = max(1, min(bh, (256 << 20) // head))
-        pooled = bh * M * 4 + 2 * bh * M * d * 2 + bh * M * 4 + 2 * 3 * bh * M * d * 2
+        # fixup lists (two), per-query log2 denominators, bf16 kbar / vsum,
+        # threshold row counts, three-part splits of qbar and kbar
+        pooled = 2 * bh * M * 4 + bh * M * 64 * 4 + 2 * bh * M * d * 2 + bh * M * 4 + 2 * 3 * bh * M * d * 2
         masks = bh * M * (-(-M // 32)) * 4
-        return pooled + masks + heads * head
+        # first-order mode: w per query, and one d x d partial per (head,
+        # chunk of blocks), chunks sized for up to 256 SMs (2 CTAs each)
+        want = min(M, max(1, -(-512 // bh)))
+        per = -(-M // want)
+        chunks = -(-M // per)
+        hyd = bh * M * 64 * 4 + bh * chunks * d * d * 4
+        return pooled + masks + hyd + heads * head
 
     for B, H, M, d in ((1, 12, 512, 128), (1, 8, 2048, 128), (1, 24, 1024, 64), (1, 2, 8192, 64),
                        (1, 1, 16384, 64), (2, 3, 37, 64)):
         got = psa.psa_workspace_size(B, H, M * 64, d)
         want = parts(B, H, M, d)
-        # each region is rounded up to 256 bytes (header + 8 regions)
-        assert want <= got <= want + 256 * 10, (B, H, M, d, got, want)
+        # each region is rounded up to 256 bytes (header + 12 regions)
+        assert want <= got <= want + 256 * 14, (B, H, M, d, got, want)
     # two heads of M = 8192 do not fit 256 MB together: one head's matrix is held
     one = psa.psa_workspace_size(1, 1, 8192 * 64, 64)
     two = psa.psa_workspace_size(1, 2, 8192 * 64, 64)

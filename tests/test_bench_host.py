@@ -61,13 +61,14 @@ def test_dense_flops_formula():
 
 def test_launches_per_step_matches_the_launch_lists():
     # launch lists of one step (pool, split3, score_tc, selection, stats_to_bf16,
-    # attention, fixup; + scan and compaction for the threshold routers)
-    assert bench.launches_per_step(1, 12, 512, "topk", False) == 7
-    assert bench.launches_per_step(1, 12, 512, "thresh", False) == 9
-    assert bench.launches_per_step(1, 8, 2048, "thresh", False) == 9      # 8 x 16 MB of scores: one batch
-    assert bench.launches_per_step(1, 1, 16384, "topk", False) == 7
-    assert bench.launches_per_step(1, 2, 16384, "topk", False) == 9       # 1 GB per head: two batches
-    assert bench.launches_per_step(1, 12, 512, "topk", True) == 3
+    # attention, its rerun of flagged blocks, fixup; + scan and compaction for
+    # the threshold routers)
+    assert bench.launches_per_step(1, 12, 512, "topk", False) == 8
+    assert bench.launches_per_step(1, 12, 512, "thresh", False) == 10
+    assert bench.launches_per_step(1, 8, 2048, "thresh", False) == 10      # 8 x 16 MB of scores: one batch
+    assert bench.launches_per_step(1, 1, 16384, "topk", False) == 8
+    assert bench.launches_per_step(1, 2, 16384, "topk", False) == 10       # 1 GB per head: two batches
+    assert bench.launches_per_step(1, 12, 512, "topk", True) == 4
 
 
 def test_reference_arm_prints_its_line_on_the_host():
