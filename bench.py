@@ -478,6 +478,83 @@ def gpu_arm(args):
         dist.destroy_process_group()
 
 
+def bwd_arm(args):
+    """The backward of the 0th-order attention (psa_attn_bwd) on the
+    workload's own block lists: pool, route and attention run once to give
+    out and lse, dout is a seeded N(0, 1) tensor, and each timed step is one
+    psa_attn_bwd call on inputs resident in HBM (L2 flushed between steps,
+    outside the events).  FLOPs: 2.5x the forward's (five products per
+    listed key pair and per pseudo-key instead of two: the scores and dP
+    recomputed, dq, dk, dv / dkbar, dvsum)."""
+    world, rank, local = _dist_setup()
+    device = torch.device("cuda", local)
+    st = Step(args.workload, args.density, seed=rank, device=device)
+    if st.dense:
+        raise SystemExit("--bwd times the routed path")
+    st.run()
+    qbar, kbar, vsum = st.stats
+    out, lse = psa.psa_attn(st.q, st.k, st.v, kbar, vsum, st.csr[0], st.csr[1], st.causal, ws=st.ws,
+                            want_lse=True, row_max=st.csr[3])
+    gen = torch.Generator(device=device).manual_seed(1000 + rank)
+    dout = torch.randn(st.q.shape, generator=gen, device=device).to(torch.bfloat16)
+    grads = tuple(torch.empty_like(st.q) for _ in range(3))
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def call():
+        psa.psa_attn_bwd(st.q, st.k, st.v, kbar, vsum, st.csr[0], st.csr[1], out, lse, dout, st.causal,
+                         ws=st.ws, grads=grads)
+
+    for _ in range(args.warmup):
+        call()
+        _flush(flush)
+    torch.cuda.synchronize()
+    status = psa.psa_read_status(st.ws)
+    rp = st.csr[0].cpu().numpy()
+    fwd_ex = executed_flops(rp, None, st.B, st.H, st.M, st.d, st.causal)
+    ex = 2.5 * fwd_ex
+    de = 2.5 * dense_flops(st.B, st.H, st.N, st.d, st.causal)
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    for i in range(args.steps):
+        evs[i][0].record(s)
+        call()
+        evs[i][1].record(s)
+        _flush(flush)
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk = clocks.stop()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world) / args.steps
+    peaks = _peaks()
+    achieved = ex / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC + " (backward of psa_attn)",
+        "value": round(weak_scaling_value(de, world, ms), 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator, seed = rank)",
+        "config": {"workload": st.name, "B": st.B, "H": st.H, "N": st.N, "d": st.d, "block": 64,
+                   "causal": st.causal, "routing": f"{st.mode} {st.param}", "variant": "backward (psa_attn_bwd)",
+                   "l2": "flushed between steps (512 MB write outside the timed events)"},
+        "roofline": {"bound": "tensor", "kernel": "bwd_pseudo + bwd_dq + bwd_dkdv (psa_attn_bwd call)",
+                     "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                     "peak_source": peaks["source"] + " bf16 burst"},
+        "flops": {"dense_equivalent": de, "executed": ex},
+        "device_status": status,
+        "gpu_launches": 7 * args.steps,  # bf16 statistics, delta, bitmaps, pseudo + its reduction, dq, dk/dv
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
 def recorded_traffic(workload: str):
     """DRAM bytes per attention launch of this workload from the ncu record
     ``profiles/traffic.json`` (dram__bytes_read.sum + dram__bytes_write.sum of
@@ -637,6 +714,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dense", action="store_true", help="time psa_dense (density 1, every block exact) instead")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward (psa_attn_bwd) on the workload's block lists instead")
     ap.add_argument("--hyd", action="store_true",
                     help="time the first-order variant (psa_hyd_stat + psa_attn_hyd) instead of psa_attn")
     args = ap.parse_args(argv)
@@ -644,6 +723,8 @@ def main(argv=None):
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         reference_arm(args)
+    elif args.bwd:
+        bwd_arm(args)
     else:
         gpu_arm(args)
 

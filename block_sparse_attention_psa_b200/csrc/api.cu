@@ -40,6 +40,8 @@ WorkspaceLayout workspace_layout(long long BH, long long M, long long d) {
   o += align256(static_cast<size_t>(BH * M * 64) * 4);
   L.hyd_partial = o;
   o += align256(psa::hyd_partial_bytes(static_cast<int>(BH), static_cast<int>(M), static_cast<int>(d)));
+  L.bwd_part = o;
+  o += 2 * align256(psa::bwd_partial_bytes(static_cast<int>(BH), static_cast<int>(M), static_cast<int>(d)));
   // block scores of as many heads as fit 256 MB (at least one)
   const size_t head_scores = static_cast<size_t>(M) * score_stride(static_cast<int>(M)) * 4;
   const long long fit = static_cast<long long>((size_t(256) << 20) / head_scores);
@@ -351,6 +353,65 @@ int psa_attn_hyd(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, 
   if (!hstat) return PSA_ERR_ARG;
   return attn_common(q, k, v, kbar, vsum, hstat, row_ptr, col_idx, col_capacity, row_max, B, H, N, d, block_size,
                      causal, out, lse, workspace, workspace_bytes, stream);
+}
+
+int psa_attn_bwd(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar,
+                 const float* vsum, const int* row_ptr, const int* col_idx, size_t col_capacity, int B, int H, int N,
+                 int d, int block_size, int causal, const psa_bf16_t* out, const float* lse, const psa_bf16_t* dout,
+                 psa_bf16_t* dq, psa_bf16_t* dk, psa_bf16_t* dv, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  if (!q || !k || !v || !kbar || !vsum || !row_ptr || !col_idx || !out || !lse || !dout || !dq || !dk || !dv ||
+      !workspace)
+    return PSA_ERR_ARG;
+  int s = check_shape(B, H, N, d, block_size);
+  if (s != PSA_OK) return s;
+  if (causal != 0 && causal != 1) return PSA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kbar) || !aligned16(vsum) || !aligned16(out) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PSA_ERR_ARG;
+  const long long bh = static_cast<long long>(B) * H;
+  const int M = N / kBlock;
+  const psa::WorkspaceLayout L = psa::workspace_layout(bh, M, d);
+  if (workspace_bytes < L.total) return PSA_ERR_CAPACITY;
+  if ((s = check_device({q, dout, dq, workspace})) != PSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
+  uint16_t* kb16 = reinterpret_cast<uint16_t*>(ws + L.kbar_bf16);
+  uint16_t* vb16 = reinterpret_cast<uint16_t*>(ws + L.vsum_bf16);
+  if (psa::launch_stats_to_bf16(kbar, vsum, bh * M * d, kb16, vb16, st) != cudaSuccess) return PSA_ERR_CUDA;
+  psa::BwdLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.kbar_bf16 = kb16;
+  a.vsum_bf16 = vb16;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.col_cap = col_capacity > static_cast<size_t>(LLONG_MAX) ? LLONG_MAX : static_cast<long long>(col_capacity);
+  a.out = out;
+  a.lse = lse;
+  a.dout = dout;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.BH = static_cast<int>(bh);
+  a.N = N;
+  a.M = M;
+  a.d = d;
+  a.causal = causal;
+  a.status = reinterpret_cast<int*>(ws);
+  // scratch of the backward: regions the forward calls use only within a call
+  a.bits = reinterpret_cast<uint32_t*>(ws + L.row_bits);
+  a.nlse2 = reinterpret_cast<float*>(ws + L.row_lse2);
+  a.delta = reinterpret_cast<float*>(ws + L.hyd_w);
+  a.dvsum = reinterpret_cast<float*>(ws + L.q_split);
+  a.dkbar = reinterpret_cast<float*>(ws + L.k_split);
+  const size_t part = (psa::bwd_partial_bytes(a.BH, M, d) + 255) & ~static_cast<size_t>(255);
+  a.part_dvs = reinterpret_cast<float*>(ws + L.bwd_part);
+  a.part_dkb = reinterpret_cast<float*>(ws + L.bwd_part + part);
+  return cuda_status(psa::launch_bwd(a, st));
 }
 
 int psa_hyd_stat(const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar, const float* vsum, int B, int H,

@@ -113,6 +113,7 @@ struct Params {
   const int* fix_src_count;
   const int* fix_src_list;
   const float* row_lse2;
+  int* sched;        // ticket counter of the dynamic unit scheduler (zero at launch)
 };
 
 // Everything every role needs to agree on about one work unit.
@@ -207,11 +208,17 @@ __device__ __forceinline__ float group_sum64(float (&v)[64], float* red, int lan
   red[gwarp * 64 + col] = v[0];
   red[gwarp * 64 + col + 1] = v[1];
   named_barrier_sync(1, 256);
+  // Warp w of one warpgroup and warp w of the other hold the same TMEM lanes
+  // of complementary tiles (the unit's even and odd tiles); which group holds
+  // which depends only on the parity the unit started at.  Adding each such
+  // pair first (IEEE addition commutes) makes the sum independent of that
+  // parity, so a unit's denominator does not depend on the units its CTA ran
+  // before it.
   float r = 0.f;
   if (gtid < 64) {
-    r = red[gtid];
+    r = red[gtid] + red[4 * 64 + gtid];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) r += red[w * 64 + gtid];
+    for (int w = 1; w < 4; ++w) r += red[w * 64 + gtid] + red[(w + 4) * 64 + gtid];
   }
   return r;
 }
@@ -288,10 +295,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_full = bars + 16;   // last GEMM2 of the unit done   (commit)
   uint64_t* o_empty = bars + 18;  // O^T read by the epilogue      (4 warps)
   uint64_t* drain = bars + 20;    // [2] teardown of the two issuers
+  uint64_t* unit_full = bars + 22;   // [4] a unit id published by the scheduler (warp 0)
+  uint64_t* unit_empty = bars + 26;  // [4] the unit id read by its four consumers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* unit_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   volatile int* stop_s = reinterpret_cast<volatile int*>(tmem_slot + 3);
+  volatile int* uring = reinterpret_cast<volatile int*>(tmem_slot + 4);   // [4] unit ids in flight
+  volatile int* next_s = reinterpret_cast<volatile int*>(tmem_slot + 8);  // softmax: the next unit
   float* red = reinterpret_cast<float*>(smem + C::kOffMisc + 512);  // [8][128] + [8]
   float* qbs = red + 8 * 128 + 8;  // block mean of the unit's queries [128]
   float* invl = qbs + 128;
@@ -304,6 +315,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   // first pass's list (unit ids from it)
   const int units = FIX ? *p.fix_src_count : p.units;
   auto uid = [&](int u) { return FIX ? __ldg(p.fix_src_list + u) : u; };
+  // Dynamic unit scheduler.  A CTA's first unit is blockIdx.x; each later one
+  // is the next ticket of the launch's counter (after the grid's first
+  // units), so CTAs that drew short units take more of them and the tail of
+  // the launch stays short.  The key producer (warp 0) draws the tickets and
+  // publishes the CTA's ul-th unit in slot ul % 4 of a shared ring; the value
+  // producer, both MMA issuers and the softmax group read every slot in
+  // order.  -1 ends the sequence.  Tickets follow the unit order (head-major),
+  // so concurrent CTAs still share one or two heads' K and V in L2.
+  auto publish = [&](int ul) -> int {
+    int u;
+    if (ul == 0) {
+      u = static_cast<int>(blockIdx.x) < units ? static_cast<int>(blockIdx.x) : -1;
+    } else {
+      u = static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1);
+      if (u >= units) u = -1;
+    }
+    const int slot = ul & 3;
+    if (ul >= 4 && !mbar_wait(&unit_empty[slot], ((ul >> 2) - 1) & 1, abort_flag, p.status)) return -1;
+    uring[slot] = u;
+    mbar_arrive(&unit_full[slot]);
+    return u;
+  };
+  auto fetch = [&](int ul) -> int {
+    const int slot = ul & 3;
+    if (!mbar_wait(&unit_full[slot], (ul >> 2) & 1, abort_flag, p.status)) return -1;
+    const int u = uring[slot];
+    mbar_arrive(&unit_empty[slot]);
+    return u;
+  };
   if constexpr (HYD) {
     // all-ones operand (bf16 1.0 = 0x3f80), read by the tensor core through the async proxy
     uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::kOffOnes);
@@ -324,6 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_full[i], 1);
       mbar_init(&o_empty[i], 4);   // the warps of one softmax warpgroup
       mbar_init(&drain[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&unit_full[i], 1);
+      mbar_init(&unit_empty[i], 4);  // V producer, both issuers, softmax
     }
     *abort_flag = 0;
     *unit_flag = 0;
@@ -357,8 +401,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int ld[2] = {0, 0};      // loads issued into each stage (lane 0)
     int qc = 0;
     bool ok = true;
-    int ul = 0;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+    for (int ul = 0; ok; ++ul) {
+      int u = -1;
+      if (lane == 0) u = keys ? publish(ul) : fetch(ul);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (u < 0) break;
       const Unit x = make_unit(uid(u), p);
       const int qb = ul & 1;
       if (keys && lane == 0) {
@@ -439,8 +486,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint64_t kKVStep = C::kKVBytes >> 4, kQStep = C::kQBytes >> 4;  // 16-byte units
       int sc = 0;
       bool ok = true;
-      int ul = 0;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+      for (int ul = 0; ok; ++ul) {
+        const int u = fetch(ul);
+        if (u < 0) break;
         const Unit x = make_unit(uid(u), p);
         const int qb = ul & 1;
         if (!(ok = mbar_wait(&q_full[qb], (ul >> 1) & 1, abort_flag, p.status))) break;
@@ -484,8 +532,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int sc = 0;
       int used[2] = {0, 0};  // GEMM2s issued on each buffer parity
       bool ok = true;
-      int ul = 0;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+      for (int ul = 0; ok; ++ul) {
+        const int u = fetch(ul);
+        if (u < 0) break;
         const Unit x = make_unit(uid(u), p);
         const int ob = ul & 1;
         const int g2_total = x.n_a2 + x.n_e;
@@ -658,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int na = 0, nb = 0;
     float nrmax = 0.f;
     auto load_next = [&](int un) {
-      if (un >= units) return;
+      if (un < 0) return;
       const int row = unit_row(uid(un), p);
       if (!p.dense) {
         na = __ldg(p.row_ptr + row);
@@ -667,16 +716,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.row_max) nrmax = __ldg(p.row_max + row);
     };
     const int nw_all = (p.M + 31) / 32;  // bitmap words of the widest candidate range
-    bool go = static_cast<int>(blockIdx.x) < units;
-    if (go) {
-      load_next(blockIdx.x);
-      if (gtid == 0) *stop_s = *abort_flag;
-      for (int i = gtid; i < nw_all; i += 256) bitmap[i] = 0u;
-      named_barrier_sync(1, 256);
-      go = !*stop_s;
-      if (go) prologue(blockIdx.x, na, nb, nrmax);
+    if (gtid == 0) {
+      *next_s = fetch(0);
+      *stop_s = *abort_flag;
     }
-    for (int u = blockIdx.x; go; u += gridDim.x, ++ul) {
+    for (int i = gtid; i < nw_all; i += 256) bitmap[i] = 0u;
+    named_barrier_sync(1, 256);
+    int u = *next_s;
+    bool go = u >= 0 && !*stop_s;
+    if (go) {
+      load_next(u);
+      prologue(u, na, nb, nrmax);
+    }
+    for (; go; ++ul) {
 
       // ---- A2 (unlisted pooled blocks) and E (listed blocks) tiles
       for (int t = 0; t < x.ntiles; ++t, ++sc) {
@@ -748,19 +800,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.lse) p.lse[static_cast<size_t>(x.row) * 64 + gtid] = lse2 * kLn2;
         if (!FIX) p.lse2_out[static_cast<size_t>(x.row) * 64 + gtid] = lse2;
       }
-      const bool more = u + static_cast<int>(gridDim.x) < units;
-      if (gtid == 0) *stop_s = *abort_flag;
+      if (gtid == 0) {
+        *next_s = fetch(ul + 1);  // the scheduler's next unit for this CTA (or -1)
+        *stop_s = *abort_flag;
+      }
       if ((gtid & 127) == 0) bulk_wait_read0();  // the last unit's store has read the staging tile
-      if (more && !p.dense)
+      if (!p.dense)
         for (int i = gtid; i < nw_all; i += 256) bitmap[i] = 0u;
       named_barrier_sync(1, 256);
       const int row_done = x.row;
       const bool had_a2 = x.n_a2 > 0;
+      const int u_done = u;
       // the next unit's setup overlaps the wait for this unit's last GEMM2
-      go = more && !*stop_s;
+      u = *next_s;
+      go = u >= 0 && !*stop_s;
       if (go) {
-        load_next(u + gridDim.x);
-        prologue(u + gridDim.x, na, nb, nrmax);
+        load_next(u);
+        prologue(u, na, nb, nrmax);
       }
       // the output: the warpgroup that does not own the next unit's first
       // tile writes all 64 query columns while the other goes on
@@ -816,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_commit();
           if (*unit_flag) {
             const int slot = atomicAdd(p.fixup_count, 1);
-            p.fixup_list[slot] = uid(u);
+            p.fixup_list[slot] = uid(u_done);
             *unit_flag = 0;
           }
         }
@@ -977,6 +1033,7 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   p.fix_src_count = nullptr;
   p.fix_src_list = nullptr;
   p.row_lse2 = nullptr;
+  p.sched = a.sched;
   cudaError_t e;
   if ((e = prepare_attn_kernel<D, HYD, false>(kSmem)) != cudaSuccess) return e;
   if ((e = prepare_attn_kernel<D, HYD, true>(kSmem)) != cudaSuccess) return e;
@@ -993,6 +1050,7 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   r.lse2_out = nullptr;
   r.fixup_count = a.fixup_count2;
   r.fixup_list = a.fixup_list2;
+  r.sched = a.sched + 1;
   attn_kernel<D, HYD, true><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, mkb, mvb, r);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // exact recomputation of what the rerun still flags

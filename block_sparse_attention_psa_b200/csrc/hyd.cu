@@ -419,9 +419,11 @@ __global__ void __launch_bounds__(kApplyThreads)
   }
 }
 
+// One CTA per SM (the ring holds an SM's shared memory): as many chunks of
+// key blocks per head as keep the grid within one wave.
 int stat_chunks(int BH, int M, int& per) {
   const int sms = device_sm_count();
-  int want = (2 * sms + BH - 1) / BH;
+  int want = sms / BH;
   if (want < 1) want = 1;
   if (want > M) want = M;
   per = (M + want - 1) / want;
@@ -458,7 +460,7 @@ cudaError_t launch_apply_d(const uint16_t* q, const float* hstat, const float* w
     return cudaErrorInvalidValue;
   const int ntile = (N + 127) / 128;
   const int sms = device_sm_count();
-  int want = (sms + BH - 1) / BH;
+  int want = sms / BH;  // one CTA per SM, one wave
   if (want < 1) want = 1;
   if (want > ntile) want = ntile;
   const int per = (ntile + want - 1) / want;

@@ -28,6 +28,7 @@ struct WorkspaceLayout {
   size_t k_split = 0;       // bf16 [3][B*H*M*d] (same for kbar)
   size_t hyd_w = 0;         // fp32 [B*H*N] (first-order mode: 0th-order share per query)
   size_t hyd_partial = 0;   // fp32 partial statistics of the first-order mode
+  size_t bwd_part = 0;      // fp32 partial pseudo-key gradients of the backward (two halves)
   size_t scores = 0;        // fp32 [score_heads][M][Mp] block scores of one batch of heads
   int score_heads = 0;      // heads per routing batch
   size_t total = 0;
@@ -100,6 +101,36 @@ struct AttnLaunch {
   float* hyd_w = nullptr;  // [BH * N] fp32 (hyd mode only)
 };
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t st);
+
+// bwd.cu: gradients of the 0th-order attention for fixed block lists
+struct BwdLaunch {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const uint16_t* kbar_bf16;
+  const uint16_t* vsum_bf16;
+  const int* row_ptr;
+  const int* col_idx;
+  long long col_cap;
+  const uint16_t* out;   // the forward's output
+  const float* lse;      // the forward's lse (natural log)
+  const uint16_t* dout;
+  uint16_t* dq;
+  uint16_t* dk;
+  uint16_t* dv;
+  int BH, N, M, d, causal;
+  int* status;
+  // workspace
+  uint32_t* bits;        // [BH*M][ceil(M/32)]
+  float* nlse2;          // [BH*N]
+  float* delta;          // [BH*N]
+  float* part_dvs;       // partial pseudo-key gradients
+  float* part_dkb;
+  float* dvsum;          // [BH*M*d]
+  float* dkbar;          // [BH*M*d]
+};
+size_t bwd_partial_bytes(int BH, int M, int d);
+cudaError_t launch_bwd(const BwdLaunch& a, cudaStream_t st);
 
 // hyd.cu: the first-order correction
 // partial matrices of the statistic kernel (bytes, for the workspace)

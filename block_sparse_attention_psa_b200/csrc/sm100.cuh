@@ -111,6 +111,14 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, void* smem_d
       : "memory");
 }
 
+// Bulk (non-tensor) copy global -> shared of `bytes` (multiple of 16, both
+// addresses 16-byte aligned), completing on `bar`; no multicast.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // 3-D tiled store shared -> global (bulk group): the box at element
 // coordinates (x, y, z); rows outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {

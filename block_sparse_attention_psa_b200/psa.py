@@ -32,7 +32,7 @@ PSA_ERR_DEVICE = 8
 EXPORTS = ("psa_status_string", "psa_version", "psa_workspace_size", "psa_route_capacity", "psa_pool",
            "psa_route_topk", "psa_route_thresh", "psa_attn", "psa_dense", "psa_read_status",
            "psa_attn_noalloc", "psa_route_thresh_prob", "psa_test_stall_next_attn",
-           "psa_read_fixup_count", "psa_hyd_stat", "psa_attn_hyd")
+           "psa_read_fixup_count", "psa_hyd_stat", "psa_attn_hyd", "psa_attn_bwd")
 
 _lib = None
 
@@ -59,6 +59,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "psa_read_status": (I, [P, ctypes.POINTER(I), P]),
         "psa_read_fixup_count": (I, [P, ctypes.POINTER(I), ctypes.POINTER(I), P]),
         "psa_hyd_stat": (I, [P, P, P, P, I, I, I, I, P, P, Z, P]),
+        "psa_attn_bwd": (I, [P, P, P, P, P, P, P, Z, I, I, I, I, I, I, P, P, P, P, P, P, P, Z, P]),
         "psa_attn_hyd": (I, [P, P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, Z, P]),
         "psa_test_stall_next_attn": (I, [I]),
         "psa_attn_noalloc": (I, [P, P, P, P, P, P, P, Z, P, I, I, I, I, I, I, P, P, P, P]),
@@ -328,6 +329,33 @@ def psa_attn_hyd(q, k, v, kbar, vsum, hstat, row_ptr, col_idx, causal: bool = Fa
           _ptr(col_idx), col_idx.numel(), _ptr(row_max), B, H, N, d, block_size, int(causal), _ptr(out),
           _ptr(lse), _ptr(ws), ws.numel(), _stream(stream, q))
     return (out, lse) if lse is not None else out
+
+
+def psa_attn_bwd(q, k, v, kbar, vsum, row_ptr, col_idx, out, lse, dout, causal: bool = False,
+                 block_size: int = 64, ws=None, grads=None, stream=None):
+    """Gradients (dq, dk, dv), bf16 [B, H, N, d], of the 0th-order attention
+    of psa_attn for fixed block lists, given its output ``out``, its ``lse``
+    and dL/dout ``dout``."""
+    B, H, N, d = _expect_qkv(q, k, v)
+    M = N // block_size if block_size > 0 else 0
+    _expect_attn_inputs(q, kbar, vsum, row_ptr, col_idx, None, B, H, M, d)
+    _expect("out", out, q, (B, H, N, d), torch.bfloat16)
+    _expect("dout", dout, q, (B, H, N, d), torch.bfloat16)
+    if lse is None:
+        raise ValueError("lse (float32 [B, H, N]) of the forward call is required")
+    _expect("lse", lse, q, (B, H, N), torch.float32)
+    if ws is None:
+        ws = workspace(B, H, N, d, q.device)
+    if grads is None:
+        grads = tuple(torch.empty_like(q) for _ in range(3))
+    dq, dk, dv = grads
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _expect(name, t, q, (B, H, N, d), torch.bfloat16)
+    _expect_ws(ws, q, B, H, N, d)
+    _call("psa_attn_bwd", q, _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vsum), _ptr(row_ptr), _ptr(col_idx),
+          col_idx.numel(), B, H, N, d, block_size, int(causal), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+          _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(stream, q))
+    return dq, dk, dv
 
 
 def psa_dense(q, k, v, causal: bool = False, ws=None, out=None, lse=None, want_lse: bool = False,

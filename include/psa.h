@@ -238,6 +238,34 @@ PSA_API int psa_attn_hyd(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf1
                          psa_bf16_t* out, float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * f-4. Gradients of the 0th-order attention of psa_attn for fixed block
+ * lists [PISA summary, "Minimal usage": the simplified 0th-order version
+ * supports training].  With out, lse the outputs of psa_attn on the same
+ * inputs and lists, and dout = dL/dout, it writes dq, dk, dv (bf16
+ * [B,H,N,d], fp32 accumulation):
+ *   D_i = dout_i . out_i,  p_ij = e^{z_ij - lse_i},  pi_iJ = e^{a_iJ - lse_i}
+ *   dS_ij = p_ij (dout_i . v_j - D_i)          (listed keys)
+ *   dA_iJ = pi_iJ (dout_i . vsum_J - 64 D_i)   (unlisted candidates)
+ *   dq_i = (sum_j dS_ij k_j + sum_J dA_iJ kbar_J) / sqrt(d)
+ *   dk_j = sum_i dS_ij q_i / sqrt(d) + dkbar_J / 64,  dkbar_J = sum_i dA_iJ q_i / sqrt(d)
+ *   dv_j = sum_i p_ij dout_i + dvsum_J,            dvsum_J = sum_i pi_iJ dout_i
+ * (block J of token j; the pooling spreads the pseudo-key gradients over the
+ * block's tokens).  The routing carries no gradient.  Inputs as psa_attn
+ * (kbar, vsum from psa_pool; lse float32 [B,H,N] required, dout bf16
+ * [B,H,N,d]); outputs dq, dk, dv bf16 [B,H,N,d].  A list entry that repeats
+ * a block or leaves the candidates is recorded as PSA_ERR_CSR in the
+ * workspace status word and left out.  `workspace` as psa_attn (the call
+ * resets its status word).  Errors as psa_attn.
+ */
+PSA_API int psa_attn_bwd(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v,
+                         const float* kbar, const float* vsum,
+                         const int* row_ptr, const int* col_idx, size_t col_capacity,
+                         int B, int H, int N, int d, int block_size, int causal,
+                         const psa_bf16_t* out, const float* lse, const psa_bf16_t* dout,
+                         psa_bf16_t* dq, psa_bf16_t* dk, psa_bf16_t* dv,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Dense attention (density = 1: every candidate block exact) through the
  * same tensor-core kernel: the comparison baseline [PISA summary, "first
  * check: compare dense and PISA outputs on the same seed and input";

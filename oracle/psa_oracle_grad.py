@@ -54,29 +54,49 @@ def _unit(q, k, v, kbar, vsum, sel, b, h, I, causal, bs):
     ez, ea = torch.exp(z - m), torch.exp(a - m)
     num = ez @ Vx + ea @ VS
     den = ez.sum(dim=1, keepdim=True) + bs * ea.sum(dim=1, keepdim=True)
-    return num / den
+    return num / den, (m + torch.log(den)).squeeze(1)
 
 
-def forward(q, k, v, row_ptr, col_idx, causal: bool, block_size: int = 64):
+def forward(q, k, v, row_ptr, col_idx, causal: bool, block_size: int = 64, with_lse: bool = False):
     """The 0th-order output [B, H, N, d] as a differentiable function of
-    torch fp64 tensors q, k, v (the block lists fixed)."""
+    torch fp64 tensors q, k, v (the block lists fixed); with ``with_lse``
+    also its lse [B, H, N] (natural log of the denominator)."""
     B, H, N, d = q.shape
     bs = block_size
     M = N // bs
     kbar = k.reshape(B, H, M, bs, d).mean(dim=3)
     vsum = v.reshape(B, H, M, bs, d).sum(dim=3)
-    rows = []
+    rows, lses = [], []
     for b in range(B):
         for h in range(H):
             for I in range(M):
                 r = (b * H + h) * M + I
-                rows.append(_unit(q, k, v, kbar, vsum, col_idx[row_ptr[r]:row_ptr[r + 1]], b, h, I, causal, bs))
-    return torch.stack(rows).reshape(B, H, N, d)
+                o, l = _unit(q, k, v, kbar, vsum, col_idx[row_ptr[r]:row_ptr[r + 1]], b, h, I, causal, bs)
+                rows.append(o)
+                lses.append(l)
+    out = torch.stack(rows).reshape(B, H, N, d)
+    if with_lse:
+        return out, torch.stack(lses).reshape(B, H, N)
+    return out
 
 
-def backward(q, k, v, row_ptr, col_idx, causal: bool, dout, block_size: int = 64):
-    """(dq, dk, dv) = the gradient of sum(out * dout), as float64 numpy arrays."""
+def backward(q, k, v, row_ptr, col_idx, causal: bool, dout, block_size: int = 64, out_for_delta=None):
+    """(dq, dk, dv) = the gradient of sum(out * dout), as float64 numpy arrays.
+
+    ``out_for_delta``: the output a backward pass is given in place of the
+    exact one.  Softmax backward passes form D_i = dout_i . out_i from that
+    given output; with out' = out + e, D shifts by delta_i = dout_i . e_i, which
+    moves every score gradient by -p_ij delta_i (-b pi_iJ delta_i for a
+    pseudo-key).  Since d lse_i / d z_ij = p_ij (and b pi_iJ for a pseudo-key),
+    those gradients are exactly the gradient of
+    sum(out * dout) - sum_i delta_i lse_i with delta held constant, which is
+    what is returned then."""
     t = [torch.tensor(np.asarray(x, dtype=np.float64), requires_grad=True) for x in (q, k, v)]
-    out = forward(*t, row_ptr, col_idx, causal, block_size)
-    (out * torch.tensor(np.asarray(dout, dtype=np.float64))).sum().backward()
+    out, lse = forward(*t, row_ptr, col_idx, causal, block_size, with_lse=True)
+    g = torch.tensor(np.asarray(dout, dtype=np.float64))
+    loss = (out * g).sum()
+    if out_for_delta is not None:
+        delta = (g * (torch.tensor(np.asarray(out_for_delta, dtype=np.float64)) - out.detach())).sum(dim=-1)
+        loss = loss - (delta * lse).sum()
+    loss.backward()
     return tuple(x.grad.numpy() for x in t)

@@ -124,3 +124,35 @@ def test_planted_gradient_mistake_is_caught(monkeypatch):
                                                                             vsum.detach(), *rest))
     with pytest.raises(AssertionError):
         test_gradients_match_central_differences(False)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_given_output_backward(causal):
+    # A backward pass forms D_i = dout_i . out_i from the output it is given.
+    # With the exact output the oracle's given-output backward is the plain
+    # gradient; with out + e it shifts dq_i by exactly -tau delta_i khat_i, where
+    # delta_i = dout_i . e_i and khat_i = sum_j p_ij k_j + sum_J pi_iJ (b kbar_J)
+    # is the softmax-weighted mean key (the attention of the oracle's plain
+    # forward with the keys as values), and leaves dv unchanged.
+    rng = np.random.default_rng(11)
+    q, k, v = _inputs(12)
+    H, N, d = q.shape[1], q.shape[2], q.shape[3]
+    M = N // BS
+    rp, ci = _random_lists(H, M, causal, rng)
+    dout = rng.standard_normal(q.shape)
+    _, kbar, vsum = O.pool(q, k, v, BS)
+    out, _ = O.attention(q, k, v, kbar, vsum, rp, ci, causal, BS)
+    out = out.reshape(q.shape)
+    plain = G.backward(q, k, v, rp, ci, causal, dout, BS)
+    same = G.backward(q, k, v, rp, ci, causal, dout, BS, out_for_delta=out)
+    for a, b in zip(plain, same):
+        assert np.abs(a - b).max() < 1e-12
+    e = 1e-3 * rng.standard_normal(q.shape)
+    shifted = G.backward(q, k, v, rp, ci, causal, dout, BS, out_for_delta=out + e)
+    delta = (dout * e).sum(-1)
+    khat, _ = O.attention(q, k, k, kbar, BS * kbar, rp, ci, causal, BS)
+    khat = khat.reshape(q.shape)
+    want_dq = plain[0] - delta[..., None] * khat / np.sqrt(d)
+    assert np.abs(shifted[0] - want_dq).max() < 1e-10
+    assert np.abs(shifted[2] - plain[2]).max() < 1e-12
+    assert np.abs(shifted[1] - plain[1]).max() > 1e-6  # dk moves too
