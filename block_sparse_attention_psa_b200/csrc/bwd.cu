@@ -21,10 +21,11 @@
 // pseudo-key gradients per tile of 128 pooled keys (partial sums over ranges
 // of query blocks, then a fixed-order reduction), dq per query block, and dk,
 // dv per key block.  The three gradient kernels run on the tensor cores
-// (tcgen05, TMEM accumulators, TMA operands) with one layout: warps 0-3 read
-// and write TMEM rows (one lane quarter each) and do the elementwise work,
-// warp 4 loads by TMA, warp 5 issues the MMAs and owns TMEM.  Every product
-// keeps M = 128 rows:
+// (tcgen05, TMEM accumulators, TMA operands) with one layout: warps 0-7 read
+// and write TMEM rows and do the elementwise work (warps w and w + 4 share
+// lane quarter w % 4, each taking half of a row's 64 columns), warp 8 loads
+// by TMA, warp 9 issues the MMAs and owns TMEM.  Every product keeps M = 128
+// rows:
 //   pseudo: S^T = Kbar_t Q_I^T, dP^T = Vsum_t dO_I^T   [128 pooled keys x 64 q]
 //           dVsum_t += Pi^T dO_I, dKbar_t += dA^T Q_I   [128 x d]
 //   dq:     S^T = K_t Q_I^T, dP^T = V_t dO_I^T           [128 keys x 64 q]
@@ -40,7 +41,8 @@
 namespace psa {
 namespace {
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdThreads = 320;  // warps 0-7 elementwise, 8 TMA, 9 MMA + TMEM
+constexpr int kWarpTma = 8, kWarpMma = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdArgs {
@@ -56,18 +58,13 @@ struct BwdArgs {
   int* status;
 };
 
-// 64 bf16 of one 128-byte row of a 128-byte-swizzled tile (row r, 16-byte
-// chunk c at (c ^ (r % 8)) * 16)
-__device__ __forceinline__ void store_row64(uint8_t* tile, int r, const uint32_t (&pk)[32]) {
+// 32 bf16 (columns 32*half ..) of row r of a 128-byte-swizzled tile (row r,
+// 16-byte chunk c at (c ^ (r % 8)) * 16)
+__device__ __forceinline__ void store_half_row(uint8_t* tile, int r, int half, const uint32_t (&pk)[16]) {
   const uint32_t base = smem_u32(tile) + r * 128;
 #pragma unroll
-  for (int c = 0; c < 8; ++c)
-    st_shared_v4(base + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-}
-
-__device__ __forceinline__ void ld_row64(uint32_t taddr, float (&v)[64]) {
-  tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(&v[0]));
-  tmem_ld32(taddr + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+  for (int c = 0; c < 4; ++c)
+    st_shared_v4(base + (((4 * half + c) ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
 }
 
 // Bounded wait for a copy's completion during teardown (ignores the abort flag).
@@ -164,7 +161,7 @@ struct PseudoCfg {
 // Item = (head, tile of 128 pooled keys, range of query blocks): partial
 // dvsum and dkbar (tau applied) of the tile over the range.
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_pseudo_kernel(const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVs,
                       const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                       const BwdArgs g, int tiles, int chunks, int per, float* __restrict__ part_dvs,
@@ -202,15 +199,15 @@ __global__ void __launch_bounds__(kBwdThreads)
       mbar_init(&full[i], 1);
       mbar_init(&stage_free[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
+      mbar_init(&s_empty[i], 8);
     }
-    mbar_init(pd_full, 4);
+    mbar_init(pd_full, 8);
     mbar_init(pd_free, 1);
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -220,7 +217,7 @@ __global__ void __launch_bounds__(kBwdThreads)
   const uint32_t tbase = *tmem_slot;
   const uint32_t t_acc_vs = tbase + 256, t_acc_kb = tbase + 256 + D;
 
-  if (warp == 4) {
+  if (warp == kWarpTma) {
     if (lane == 0 && n > 0) {
       // the tile's pooled keys and value sums, once
       mbar_arrive_expect_tx(kv_full, 2 * C::kTile);
@@ -253,7 +250,7 @@ __global__ void __launch_bounds__(kBwdThreads)
         if (issued[s]) drain_wait(&full[s], (issued[s] - 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     if (lane == 0) {
       bool ok = n == 0 || mbar_wait(kv_full, 0, abort_flag, g.status);
       const uint64_t dKb = sdesc_sw128(smem_u32(sKb), 16, 1024);
@@ -300,9 +297,11 @@ __global__ void __launch_bounds__(kBwdThreads)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise
-    const int j = warp * 32 + lane;          // TMEM lane = pooled key of the tile
+    const int quarter = warp & 3, half = warp >> 2;
+    const int j = quarter * 32 + lane;       // TMEM lane = pooled key of the tile
+    const int c0 = 32 * half;                // this thread's 32 query columns
     const int J = tile * 128 + j;
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     for (int i = 0; i < n; ++i) {
       const int s = i & 1, b = i & 1;
       const int I = start + i;
@@ -311,26 +310,26 @@ __global__ void __launch_bounds__(kBwdThreads)
       mbar_wait(&full[s], (i >> 1) & 1, abort_flag, g.status);
       mbar_wait(&s_full[b], (i >> 1) & 1, abort_flag, g.status);
       tc_fence_after();
-      float sv[64], dp[64];
-      ld_row64(tbase + lane_addr + 128 * b, sv);
-      ld_row64(tbase + lane_addr + 128 * b + 64, dp);
+      float sv[32], dp[32];
+      tmem_ld32(tbase + lane_addr + 128 * b + c0, sv);
+      tmem_ld32(tbase + lane_addr + 128 * b + 64 + c0, dp);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[b]);
-      const float* nl = reinterpret_cast<const float*>(smem + C::kOffStage + s * C::kStage + 2 * C::kQ);
+      const float* nl = reinterpret_cast<const float*>(smem + C::kOffStage + s * C::kStage + 2 * C::kQ) + c0;
       const float* dl = nl + 64;
-      uint32_t pi[32], da[32];
+      uint32_t pi[16], da[16];
 #pragma unroll
-      for (int q = 0; q < 64; q += 2) {
+      for (int q = 0; q < 32; q += 2) {
         float e0 = valid ? ex2_approx(fmaf(sv[q], g.sl, nl[q])) : 0.f;
         float e1 = valid ? ex2_approx(fmaf(sv[q + 1], g.sl, nl[q + 1])) : 0.f;
         pi[q / 2] = pack_bf16x2(e0, e1);
         da[q / 2] = pack_bf16x2(e0 * (dp[q] - 64.f * dl[q]), e1 * (dp[q + 1] - 64.f * dl[q + 1]));
       }
       if (i >= 1) mbar_wait(pd_free, (i - 1) & 1, abort_flag, g.status);
-      store_row64(sPi, j, pi);
-      store_row64(sDa, j, da);
+      store_half_row(sPi, j, half, pi);
+      store_half_row(sDa, j, half, da);
       fence_async_shared();
       __syncwarp();
       if (lane == 0) mbar_arrive(pd_full);
@@ -341,7 +340,7 @@ __global__ void __launch_bounds__(kBwdThreads)
     float* dvs = part_dvs + (static_cast<size_t>(item) * 128 + j) * D;
     float* dkb = part_dkb + (static_cast<size_t>(item) * 128 + j) * D;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {  // this half's D/2 features
       float a[32], k[32];
       if (n > 0 && ok) {
         tmem_ld32(t_acc_vs + lane_addr + 32 * c, a);
@@ -361,7 +360,7 @@ __global__ void __launch_bounds__(kBwdThreads)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
@@ -390,16 +389,26 @@ __global__ void __launch_bounds__(256) bwd_pseudo_reduce_kernel(const float* __r
 }
 
 // ------------------------------------------------------------------ dq
+// A unit is one query block: its steps are the forward's tile stream (pooled
+// tiles of 128 unlisted candidates, then pairs of listed blocks).  The key
+// rows of a step stay in shared memory until dq^T += K^T dS^T has read them,
+// after the elementwise work, so they get a 3-slot ring; the value rows are
+// free once dP^T is issued (2 slots); q and dO of a unit have one stage
+// (released when its last S^T / dP^T is done) and its -lse log2e and D two
+// small slots (released by the elementwise warps).  The MMA warp issues
+// whichever of "scores of the next step" and "dq of the oldest step" is ready.
 template <int D>
 struct DqCfg {
   static constexpr int kQ = 64 * D * 2;
-  static constexpr int kUnit = (2 * kQ + 512 + 1023) / 1024 * 1024;  // q, dO, -lse log2e, D
-  static constexpr int kTile = 128 * D * 2;                           // 128 key rows (K or Kbar)
-  static constexpr int kStep = 2 * kTile;                             // + the V (or Vsum) rows
-  static constexpr int kOffStep = 2 * kUnit;
-  static constexpr int kOffDs = kOffStep + 2 * kStep;
-  static constexpr int kOffBars = kOffDs + 128 * 128;
+  static constexpr int kTile = 128 * D * 2;  // 128 key (or value) rows
+  static constexpr int kKSlots = 3, kVSlots = 2;
+  static constexpr int kOffK = 2 * kQ;                     // q, dO at 0, kQ
+  static constexpr int kOffV = kOffK + kKSlots * kTile;
+  static constexpr int kOffDs = kOffV + kVSlots * kTile;
+  static constexpr int kOffNl = kOffDs + 128 * 128;         // [2][-lse log2e 64, D 64]
+  static constexpr int kOffBars = kOffNl + 2 * 512;
   static constexpr int kSmem = kOffBars + 256 + 1024;
+  static_assert(kSmem <= 232448, "shared memory of one CTA");
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);
   // dq^T [D x 64 q] += K^T (A: M = features, MN-major) . dS^T (B: N = q, MN-major)
   static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 64, 1, 1);
@@ -432,7 +441,7 @@ __device__ __forceinline__ DqUnit dq_unit(int u, const BwdArgs& g) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVs,
@@ -442,18 +451,21 @@ __global__ void __launch_bounds__(kBwdThreads)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sDs = smem + C::kOffDs;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
-  uint64_t* u_full = bars + 0;     // [2] q, dO, lse, D of a unit landed
-  uint64_t* u_free = bars + 2;     // [2] the unit's MMAs are done
-  uint64_t* t_full = bars + 4;     // [2] a step's key / value rows landed
-  uint64_t* t_free = bars + 6;     // [2] the step's MMAs are done
-  uint64_t* s_full = bars + 8;     // [2] S^T, dP^T ready
-  uint64_t* s_empty = bars + 10;   // [2] read by the 4 elementwise warps
-  uint64_t* ds_full = bars + 12;   // dS^T written (4 warps)
-  uint64_t* ds_free = bars + 13;   // its MMA is done
-  uint64_t* dq_full = bars + 14;   // [2] a unit's dq^T is complete
-  uint64_t* dq_empty = bars + 16;  // [2] read by the 4 elementwise warps
-  uint64_t* drain = bars + 18;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  uint64_t* u_full = bars + 0;     // [2] by unit parity: q, dO, -lse log2e, D landed
+  uint64_t* u_free = bars + 2;     // q, dO stage: the unit's last S^T / dP^T done
+  uint64_t* nl_free = bars + 3;    // [2] -lse log2e, D slot read by the 8 elementwise warps
+  uint64_t* k_full = bars + 5;     // [3] key rows of a step landed
+  uint64_t* k_free = bars + 8;     // [3] the step's dq MMA is done
+  uint64_t* v_full = bars + 11;    // [2] value rows landed
+  uint64_t* v_free = bars + 13;    // [2] the step's dP^T is done
+  uint64_t* s_full = bars + 15;    // [2] S^T, dP^T ready
+  uint64_t* s_empty = bars + 17;   // [2] read by the 8 elementwise warps
+  uint64_t* ds_full = bars + 19;   // dS^T written (8 warps)
+  uint64_t* ds_free = bars + 20;   // its MMA is done
+  uint64_t* dq_full = bars + 21;   // [2] a unit's dq^T is complete
+  uint64_t* dq_empty = bars + 23;  // [2] read by the 8 elementwise warps
+  uint64_t* drain = bars + 25;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -461,21 +473,26 @@ __global__ void __launch_bounds__(kBwdThreads)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&u_full[i], 1);
-      mbar_init(&u_free[i], 1);
-      mbar_init(&t_full[i], 1);
-      mbar_init(&t_free[i], 1);
+      mbar_init(&nl_free[i], 8);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_free[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
+      mbar_init(&s_empty[i], 8);
       mbar_init(&dq_full[i], 1);
-      mbar_init(&dq_empty[i], 4);
+      mbar_init(&dq_empty[i], 8);
     }
-    mbar_init(ds_full, 4);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_free[i], 1);
+    }
+    mbar_init(u_free, 1);
+    mbar_init(ds_full, 8);
     mbar_init(ds_free, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -484,30 +501,29 @@ __global__ void __launch_bounds__(kBwdThreads)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kWarpTma) {
+    // ---------------------------------------------------------- producer
     if (lane == 0) {
-      int sc = 0, ul = 0;
-      int un_issued[2] = {0, 0}, st_issued[2] = {0, 0};
+      int si = 0, ul = 0;
+      int k_iss[3] = {0, 0, 0}, v_iss[2] = {0, 0}, u_iss[2] = {0, 0};
       bool ok = true;
       for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++ul) {
         const DqUnit x = dq_unit(u, g);
         const int ub = ul & 1;
-        if (ul >= 2 && !(ok = mbar_wait(&u_free[ub], ((ul >> 1) - 1) & 1, abort_flag, g.status))) break;
-        uint8_t* us = smem + ub * C::kUnit;
+        // q, dO stage: the previous unit's scores are done; its -lse / D slot: read
+        if (ul >= 1 && !(ok = mbar_wait(u_free, (ul - 1) & 1, abort_flag, g.status))) break;
+        if (ul >= 2 && !(ok = mbar_wait(&nl_free[ub], ((ul >> 1) - 1) & 1, abort_flag, g.status))) break;
         mbar_arrive_expect_tx(&u_full[ub], 2 * C::kQ + 512);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(&tmQ, us + c * 8192, &u_full[ub], 64 * c, 64 * x.I, x.bh);
-          tma_load_3d(&tmDO, us + C::kQ + c * 8192, &u_full[ub], 64 * c, 64 * x.I, x.bh);
+          tma_load_3d(&tmQ, smem + c * 8192, &u_full[ub], 64 * c, 64 * x.I, x.bh);
+          tma_load_3d(&tmDO, smem + C::kQ + c * 8192, &u_full[ub], 64 * c, 64 * x.I, x.bh);
         }
         const size_t r0 = static_cast<size_t>(x.bh) * g.N + 64 * x.I;
-        bulk_load(us + 2 * C::kQ, g.nlse2 + r0, 256, &u_full[ub]);
-        bulk_load(us + 2 * C::kQ + 256, g.delta + r0, 256, &u_full[ub]);
-        ++un_issued[ub];
-        for (int t = 0; t < x.ntiles; ++t, ++sc) {
-          const int ts = sc & 1;
-          if (sc >= 2 && !(ok = mbar_wait(&t_free[ts], ((sc >> 1) - 1) & 1, abort_flag, g.status))) break;
-          uint8_t* st = smem + C::kOffStep + ts * C::kStep;
+        bulk_load(smem + C::kOffNl + ub * 512, g.nlse2 + r0, 256, &u_full[ub]);
+        bulk_load(smem + C::kOffNl + ub * 512 + 256, g.delta + r0, 256, &u_full[ub]);
+        ++u_iss[ub];
+        for (int t = 0; ok && t < x.ntiles; ++t, ++si) {
           const CUtensorMap *mk, *mv;
           int y0, y1;
           if (t < x.n_a2) {
@@ -526,71 +542,122 @@ __global__ void __launch_bounds__(kBwdThreads)
             y0 = 64 * j1;
             y1 = 64 * j2;
           }
-          mbar_arrive_expect_tx(&t_full[ts], C::kStep);
+          const int ks = si % 3, vs = si & 1;
+          if (si >= 3 && !(ok = mbar_wait(&k_free[ks], ((si / 3) - 1) & 1, abort_flag, g.status))) break;
+          uint8_t* kd = smem + C::kOffK + ks * C::kTile;
+          mbar_arrive_expect_tx(&k_full[ks], C::kTile);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d(mk, st + c * 16384, &t_full[ts], 64 * c, y0, x.bh);
-            tma_load_3d(mk, st + c * 16384 + 8192, &t_full[ts], 64 * c, y1, x.bh);
-            tma_load_3d(mv, st + C::kTile + c * 16384, &t_full[ts], 64 * c, y0, x.bh);
-            tma_load_3d(mv, st + C::kTile + c * 16384 + 8192, &t_full[ts], 64 * c, y1, x.bh);
+            tma_load_3d(mk, kd + c * 16384, &k_full[ks], 64 * c, y0, x.bh);
+            tma_load_3d(mk, kd + c * 16384 + 8192, &k_full[ks], 64 * c, y1, x.bh);
           }
-          ++st_issued[ts];
+          ++k_iss[ks];
+          if (si >= 2 && !(ok = mbar_wait(&v_free[vs], ((si >> 1) - 1) & 1, abort_flag, g.status))) break;
+          uint8_t* vd = smem + C::kOffV + vs * C::kTile;
+          mbar_arrive_expect_tx(&v_full[vs], C::kTile);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d(mv, vd + c * 16384, &v_full[vs], 64 * c, y0, x.bh);
+            tma_load_3d(mv, vd + c * 16384 + 8192, &v_full[vs], 64 * c, y1, x.bh);
+          }
+          ++v_iss[vs];
         }
       }
+      for (int b = 0; b < 3; ++b)
+        if (k_iss[b]) drain_wait(&k_full[b], (k_iss[b] - 1) & 1);
       for (int b = 0; b < 2; ++b) {
-        if (un_issued[b]) drain_wait(&u_full[b], (un_issued[b] - 1) & 1);
-        if (st_issued[b]) drain_wait(&t_full[b], (st_issued[b] - 1) & 1);
+        if (v_iss[b]) drain_wait(&v_full[b], (v_iss[b] - 1) & 1);
+        if (u_iss[b]) drain_wait(&u_full[b], (u_iss[b] - 1) & 1);
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
+    // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint64_t dUnit = sdesc_sw128(smem_u32(smem), 16, 1024);
-      const uint64_t dStep = sdesc_sw128(smem_u32(smem + C::kOffStep), 16, 1024);
+      const uint64_t dQ = sdesc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t dO = sdesc_sw128(smem_u32(smem + C::kQ), 16, 1024);
+      const uint64_t dK = sdesc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
+      const uint64_t dV = sdesc_sw128(smem_u32(smem + C::kOffV), 16, 1024);
       // key rows as the MN-major A of dq^T: M = features (64-feature atoms 16 KB apart)
-      const uint64_t dStepMN = sdesc_sw128(smem_u32(smem + C::kOffStep), D == 128 ? 16384 : 0, 1024);
+      const uint64_t dKmn = sdesc_sw128(smem_u32(smem + C::kOffK), D == 128 ? 16384 : 0, 1024);
       const uint64_t dDs = sdesc_sw128(smem_u32(sDs), 16, 1024);
-      constexpr uint64_t kU16 = C::kUnit >> 4, kQ16 = C::kQ >> 4, kS16 = C::kStep >> 4, kT16 = C::kTile >> 4;
-      int sc = 0, ul = 0;
+      constexpr uint64_t kT16 = C::kTile >> 4;
+      // the steps whose dq MMA is pending (at most two: one S^T buffer each)
+      struct Pending {
+        int ul, first, last;  // the step's unit (by CTA-local index), first / last step of it
+      } pend[2];
+      int ul_s = 0, t_s = 0, si_s = 0, si_a = 0;
+      int u_s = blockIdx.x;
+      DqUnit xs;
+      if (u_s < units) xs = dq_unit(u_s, g);
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++ul) {
-        const DqUnit x = dq_unit(u, g);
-        const int ub = ul & 1;
-        if (!(ok = mbar_wait(&u_full[ub], (ul >> 1) & 1, abort_flag, g.status))) break;
-        if (ul >= 2 && !(ok = mbar_wait(&dq_empty[ub], ((ul >> 1) - 1) & 1, abort_flag, g.status))) break;
-        const uint64_t q = dUnit + ub * kU16, o = q + kQ16;
-        const uint32_t t_dq = tbase + 256 + 64 * ub;
-        for (int t = 0; ok && t <= x.ntiles; ++t) {
-          if (t < x.ntiles) {
-            const int ts = (sc + t) & 1, b = ts;
-            const int si = sc + t;
-            if (!(ok = mbar_wait(&t_full[ts], (si >> 1) & 1, abort_flag, g.status))) break;
-            if (si >= 2 && !(ok = mbar_wait(&s_empty[b], ((si >> 1) - 1) & 1, abort_flag, g.status))) break;
+      long long idle_since = clock64();
+      while (ok && (u_s < units || si_a < si_s)) {
+        bool progress = false;
+        // scores of the next step
+        if (u_s < units && si_s - si_a < 2) {
+          const int ub = ul_s & 1, ks = si_s % 3, vs = si_s & 1, b = si_s & 1;
+          if (mbar_try_wait(&u_full[ub], (ul_s >> 1) & 1) && mbar_try_wait(&k_full[ks], (si_s / 3) & 1) &&
+              mbar_try_wait(&v_full[vs], (si_s >> 1) & 1) &&
+              (si_s < 2 || mbar_try_wait(&s_empty[b], ((si_s >> 1) - 1) & 1))) {
             tc_fence_after();
-            const uint64_t kt = dStep + ts * kS16, vt = kt + kT16;
+            const uint64_t kt = dK + ks * kT16, vt = dV + vs * kT16;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint64_t ka = (kk >> 2) * 1024 + (kk & 3) * 2, kb = (kk >> 2) * 512 + (kk & 3) * 2;
-              tc_mma_bf16(tbase + 128 * b, kt + ka, q + kb, C::kIdescS, kk > 0 ? 1u : 0u);
-              tc_mma_bf16(tbase + 128 * b + 64, vt + ka, o + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+              tc_mma_bf16(tbase + 128 * b, kt + ka, dQ + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+              tc_mma_bf16(tbase + 128 * b + 64, vt + ka, dO + kb, C::kIdescS, kk > 0 ? 1u : 0u);
             }
             tc_commit(&s_full[b]);
-          }
-          if (t >= 1) {
-            const int si = sc + t - 1, ts = si & 1;
-            if (!(ok = mbar_wait(ds_full, si & 1, abort_flag, g.status))) break;
-            tc_fence_after();
-            const uint64_t a = dStepMN + ts * kS16;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // K = 128 key rows
-              tc_mma_bf16(t_dq, a + 128 * kk, dDs + 128 * kk, C::kIdescAcc, (t > 1 || kk > 0) ? 1u : 0u);
-            tc_commit(ds_free);
-            tc_commit(&t_free[ts]);
+            tc_commit(&v_free[vs]);
+            const bool last = t_s == xs.ntiles - 1;
+            if (last) tc_commit(u_free);
+            pend[si_s & 1] = {ul_s, t_s == 0, last};
+            ++si_s;
+            if (last) {
+              ++ul_s;
+              t_s = 0;
+              u_s += gridDim.x;
+              if (u_s < units) xs = dq_unit(u_s, g);
+            } else {
+              ++t_s;
+            }
+            progress = true;
           }
         }
-        sc += x.ntiles;
-        tc_commit(&dq_full[ub]);
-        tc_commit(&u_free[ub]);
+        // dq of the oldest pending step
+        if (si_a < si_s) {
+          const Pending pa = pend[si_a & 1];
+          const int ub = pa.ul & 1;
+          if (mbar_try_wait(ds_full, si_a & 1)) {
+            // the unit's first dq MMA overwrites dq^T[ub]: the epilogue of the unit
+            // two before (same buffer) must have read it
+            const bool free_buf =
+                !pa.first || pa.ul < 2 || mbar_try_wait(&dq_empty[ub], ((pa.ul >> 1) - 1) & 1);
+            if (free_buf) {
+              tc_fence_after();
+              const uint32_t t_dq = tbase + 256 + 64 * ub;
+              const uint64_t a = dKmn + (si_a % 3) * kT16;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)  // K = 128 key rows
+                tc_mma_bf16(t_dq, a + 128 * kk, dDs + 128 * kk, C::kIdescAcc, (!pa.first || kk > 0) ? 1u : 0u);
+              tc_commit(ds_free);
+              tc_commit(&k_free[si_a % 3]);
+              if (pa.last) tc_commit(&dq_full[ub]);
+              ++si_a;
+              progress = true;
+            }
+          }
+        }
+        if (progress) {
+          idle_since = clock64();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (clock64() - idle_since > kWaitCycles) {
+          *abort_flag = 1;
+          record_status(g.status, kStatusTimeout);
+          ok = false;
+        }
       }
       tc_commit(drain);
       drain_wait(drain, 0);
@@ -598,26 +665,43 @@ __global__ void __launch_bounds__(kBwdThreads)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise
-    const int r = warp * 32 + lane;  // TMEM lane: key row of S^T, feature row of dq^T
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;  // TMEM lane: key row of S^T, feature row of dq^T
+    const int c0 = 32 * half;           // this thread's 32 query columns
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     int sc = 0, ul = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++ul) {
       const DqUnit x = dq_unit(u, g);
       const int ub = ul & 1;
       if (!mbar_wait(&u_full[ub], (ul >> 1) & 1, abort_flag, g.status)) break;
-      const float* nl = reinterpret_cast<const float*>(smem + ub * C::kUnit + 2 * C::kQ);
+      const float* nl = reinterpret_cast<const float*>(smem + C::kOffNl + ub * 512);
       const float* dl = nl + 64;
       bool stop = false;
+      // what decides this thread's row of step t: the listed-block bitmap word
+      // (pooled tile) or the listed block (exact tile); loaded a step ahead so
+      // the load's latency stays off the step's critical path
+      auto fetch_row = [&](int t) -> int {
+        if (t < x.n_a2) {
+          const int J = 128 * t + r;
+          return J < x.pcand ? static_cast<int>(__ldg(g.bits + (static_cast<size_t>(x.bh) * g.M + x.I) * g.nw +
+                                                      (J >> 5)))
+                             : -1;
+        }
+        const int idx = 2 * (t - x.n_a2) + (r >> 6);
+        return idx < x.nsel ? __ldg(g.col_idx + x.rp + idx) : -1;
+      };
+      int next_row = fetch_row(0);
       for (int t = 0; t < x.ntiles; ++t, ++sc) {
         const int b = sc & 1;
         const bool pooled = t < x.n_a2;
+        const int cur_row = next_row;
+        if (t + 1 < x.ntiles) next_row = fetch_row(t + 1);
         bool valid, diag = false;
         if (pooled) {
           const int J = 128 * t + r;
-          valid = J < x.pcand && !listed(g, x.bh, x.I, J);
+          valid = J < x.pcand && !((static_cast<uint32_t>(cur_row) >> (J & 31)) & 1u);
         } else {
-          const int idx = 2 * (t - x.n_a2) + (r >> 6);
-          const int J = idx < x.nsel ? __ldg(g.col_idx + x.rp + idx) : -1;
+          const int J = cur_row;
           valid = J >= 0 && J < x.cand;
           diag = g.causal && J == x.I;
         }
@@ -626,46 +710,46 @@ __global__ void __launch_bounds__(kBwdThreads)
           break;
         }
         tc_fence_after();
-        float sv[64], dp[64];
-        ld_row64(tbase + lane_addr + 128 * b, sv);
-        ld_row64(tbase + lane_addr + 128 * b + 64, dp);
+        float sv[32], dp[32];
+        tmem_ld32(tbase + lane_addr + 128 * b + c0, sv);
+        tmem_ld32(tbase + lane_addr + 128 * b + 64 + c0, dp);
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[b]);
         const float wD = pooled ? 64.f : 1.f;
         const int kj = r & 63;
-        uint32_t ds[32];
+        uint32_t ds[16];
 #pragma unroll
-        for (int q = 0; q < 64; q += 2) {
-          float e0 = valid ? ex2_approx(fmaf(sv[q], g.sl, nl[q])) : 0.f;
-          float e1 = valid ? ex2_approx(fmaf(sv[q + 1], g.sl, nl[q + 1])) : 0.f;
+        for (int q = 0; q < 32; q += 2) {
+          const int qq = c0 + q;
+          float e0 = valid ? ex2_approx(fmaf(sv[q], g.sl, nl[qq])) : 0.f;
+          float e1 = valid ? ex2_approx(fmaf(sv[q + 1], g.sl, nl[qq + 1])) : 0.f;
           if (diag) {
-            e0 = kj <= q ? e0 : 0.f;
-            e1 = kj <= q + 1 ? e1 : 0.f;
+            e0 = kj <= qq ? e0 : 0.f;
+            e1 = kj <= qq + 1 ? e1 : 0.f;
           }
-          ds[q / 2] = pack_bf16x2(e0 * (dp[q] - wD * dl[q]), e1 * (dp[q + 1] - wD * dl[q + 1]));
+          ds[q / 2] = pack_bf16x2(e0 * (dp[q] - wD * dl[qq]), e1 * (dp[q + 1] - wD * dl[qq + 1]));
         }
         if (sc >= 1) mbar_wait(ds_free, (sc - 1) & 1, abort_flag, g.status);
-        store_row64(sDs, r, ds);
+        store_half_row(sDs, r, half, ds);
         fence_async_shared();
         __syncwarp();
         if (lane == 0) mbar_arrive(ds_full);
       }
       if (stop) break;
-      // dq of the unit: feature row r, 64 query columns
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&nl_free[ub]);  // this unit's -lse / D slot is read
+      // dq of the unit: feature row r, this thread's 32 query columns
       if (!mbar_wait(&dq_full[ub], (ul >> 1) & 1, abort_flag, g.status)) break;
       tc_fence_after();
       if (r < D) {  // warp-uniform
-        __nv_bfloat16* dst = dq + (static_cast<size_t>(x.bh) * g.N + 64 * x.I) * D + r;
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          float v[32];
-          tmem_ld32(tbase + lane_addr + 256 + 64 * ub + 32 * h, v);
-          tc_wait_ld();
+        __nv_bfloat16* dst = dq + (static_cast<size_t>(x.bh) * g.N + 64 * x.I + c0) * D + r;
+        float v[32];
+        tmem_ld32(tbase + lane_addr + 256 + 64 * ub + c0, v);
+        tc_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) dst[static_cast<size_t>(32 * h + q) * D] = __float2bfloat16_rn(g.tau * v[q]);
-        }
+        for (int q = 0; q < 32; ++q) dst[static_cast<size_t>(q) * D] = __float2bfloat16_rn(g.tau * v[q]);
       }
       tc_fence_before();
       __syncwarp();
@@ -674,7 +758,7 @@ __global__ void __launch_bounds__(kBwdThreads)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
@@ -689,8 +773,10 @@ struct KvCfg {
   static constexpr int kOffStage = 2 * kBlk;
   static constexpr int kOffP = kOffStage + 2 * kStage;
   static constexpr int kOffDs = kOffP + 128 * 128;
-  static constexpr int kOffBars = kOffDs + 128 * 128;
+  static constexpr int kOffBal = kOffDs + 128 * 128;            // ballots of the listing scan [M / 32]
+  static constexpr int kOffBars = kOffBal + kMaxBlocks / 8;
   static constexpr int kSmem = kOffBars + 256 + 1024;
+  static_assert(kSmem <= 232448, "shared memory of one CTA");
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);    // [128 q x 64 keys]
   static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 64, 1, 1);  // [D x 64 keys] += [D x 128 q] . [128 q x 64]
 };
@@ -700,7 +786,7 @@ struct KvMeta {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const BwdArgs g, const float* __restrict__ dkbar, const float* __restrict__ dvsum,
@@ -736,17 +822,17 @@ __global__ void __launch_bounds__(kBwdThreads)
       mbar_init(&full[i], 1);
       mbar_init(&stage_free[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
+      mbar_init(&s_empty[i], 8);
     }
-    mbar_init(pd_full, 4);
+    mbar_init(pd_full, 8);
     mbar_init(pd_free, 1);
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, 8);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -758,7 +844,7 @@ __global__ void __launch_bounds__(kBwdThreads)
   auto stage = [&](int s) { return smem + C::kOffStage + s * C::kStage; };
   auto meta = [&](int s) { return reinterpret_cast<volatile KvMeta*>(stage(s) + 2 * C::kPair + 1024); };
 
-  if (warp == 4) {
+  if (warp == kWarpTma) {
     // ---------------------------------------------------------- producer
     // the query blocks that list key block J, in pairs
     int sc = 0, il = 0;
@@ -780,13 +866,29 @@ __global__ void __launch_bounds__(kBwdThreads)
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
+      // the rows that list J: one ballot per 32 rows, eight independent bitmap
+      // loads per lane in flight, the ballots kept in shared memory
       const int I0 = g.causal ? J : 0;
+      const int ngroups = (g.M - I0 + 31) / 32;
+      uint32_t* bal = reinterpret_cast<uint32_t*>(smem + C::kOffBal);
       int cnt = 0;
-      for (int gI = I0; gI < g.M; gI += 32) {
-        const int I = gI + lane;
-        const bool on = I < g.M && listed(g, bh, I, J);
-        cnt += __popc(__ballot_sync(0xffffffffu, on));
+      for (int g0 = 0; g0 < ngroups; g0 += 8) {
+        bool on[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int I = I0 + 32 * (g0 + u) + lane;
+          on[u] = g0 + u < ngroups && I < g.M && listed(g, bh, I, J);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t w = __ballot_sync(0xffffffffu, on[u]);
+          if (g0 + u < ngroups) {
+            if (lane == 0) bal[g0 + u] = w;
+            cnt += __popc(w);
+          }
+        }
       }
+      __syncwarp();
       const int nsteps = cnt == 0 ? 1 : (cnt + 1) / 2;
       int k = 0, pending = -1;
       auto emit = [&](int Ia, int Ib) {
@@ -823,21 +925,21 @@ __global__ void __launch_bounds__(kBwdThreads)
         ++sc;
         ++k;
       };
-      for (int gI = I0; gI < g.M; gI += 32) {
-        const int I = gI + lane;
-        const bool on = I < g.M && listed(g, bh, I, J);
-        uint32_t m = __ballot_sync(0xffffffffu, on);
+      for (int gi = 0; gi < ngroups; ++gi) {
+        uint32_t m = bal[gi];
         while (m) {
           const int l = __ffs(m) - 1;
           m &= m - 1;
+          const int I = I0 + 32 * gi + l;
           if (pending < 0) {
-            pending = gI + l;
+            pending = I;
           } else {
-            emit(pending, gI + l);
+            emit(pending, I);
             pending = -1;
           }
         }
       }
+      __syncwarp();
       if (pending >= 0) emit(pending, -1);
       if (cnt == 0) emit(-1, -1);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -848,7 +950,7 @@ __global__ void __launch_bounds__(kBwdThreads)
         if (st_issued[b]) drain_wait(&full[b], (st_issued[b] - 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
@@ -859,64 +961,85 @@ __global__ void __launch_bounds__(kBwdThreads)
       const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
       const uint64_t dDs = sdesc_sw128(smem_u32(sDs), 16, 1024);
       constexpr uint64_t kSt16 = C::kStage >> 4, kPair16 = C::kPair >> 4;
-      int sc = 0, il = 0;
+      // Issue whichever is ready: the scores of the next step (an S / dP
+      // buffer free, its rows landed) or the accumulation of the oldest
+      // pending step (its P and dS written), so a step's stage is released as
+      // early as its accumulation can run.
+      struct Pending {
+        int il, first, last, has;  // item (CTA-local index), first / last step of it, any rows
+      } pend[2];
+      int sc_s = 0, sc_a = 0, il_s = 0;
+      int it_s = blockIdx.x;
+      bool first_step = true;   // the next S step opens its item
+      bool acc_started = false; // an accumulation of the current item has run
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++il) {
-        if (!(ok = mbar_wait(item_full, il & 1, abort_flag, g.status))) break;
-        if (il >= 1 && !(ok = mbar_wait(acc_empty, (il - 1) & 1, abort_flag, g.status))) break;
-        bool first = true;   // next accumulation starts the item's dK^T, dV^T
-        int prev = -1;       // step whose accumulation is pending
-        bool prev_has = false;
-        for (;;) {
-          const int s = sc & 1, b = sc & 1;
-          if (!(ok = mbar_wait(&full[s], (sc >> 1) & 1, abort_flag, g.status))) break;
-          if (sc >= 2 && !(ok = mbar_wait(&s_empty[b], ((sc >> 1) - 1) & 1, abort_flag, g.status))) break;
-          volatile KvMeta* m = meta(s);
-          const bool has = m->Ia >= 0;
-          const bool last = m->last != 0;
-          tc_fence_after();
-          if (has) {
-            const uint64_t q = dSt + s * kSt16, o = q + kPair16;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t ka = (kk >> 2) * 1024 + (kk & 3) * 2, kb = (kk >> 2) * 512 + (kk & 3) * 2;
-              tc_mma_bf16(tbase + 128 * b, q + ka, dK + kb, C::kIdescS, kk > 0 ? 1u : 0u);
-              tc_mma_bf16(tbase + 128 * b + 64, o + ka, dV + kb, C::kIdescS, kk > 0 ? 1u : 0u);
-            }
-          }
-          tc_commit(&s_full[b]);
-          auto accumulate = [&](int step, bool with) {
-            const int ss = step & 1;
-            if (!(ok = mbar_wait(pd_full, step & 1, abort_flag, g.status))) return;
+      long long idle_since = clock64();
+      while (ok && (it_s < items || sc_a < sc_s)) {
+        bool progress = false;
+        if (it_s < items && sc_s - sc_a < 2) {
+          const int s = sc_s & 1, b = sc_s & 1;
+          if (mbar_try_wait(item_full, il_s & 1) && mbar_try_wait(&full[s], (sc_s >> 1) & 1) &&
+              (sc_s < 2 || mbar_try_wait(&s_empty[b], ((sc_s >> 1) - 1) & 1))) {
+            volatile KvMeta* m = meta(s);
+            const bool has = m->Ia >= 0;
+            const bool last = m->last != 0;
             tc_fence_after();
-            if (with) {
+            if (has) {
+              const uint64_t q = dSt + s * kSt16, o = q + kPair16;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t ka = (kk >> 2) * 1024 + (kk & 3) * 2, kb = (kk >> 2) * 512 + (kk & 3) * 2;
+                tc_mma_bf16(tbase + 128 * b, q + ka, dK + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+                tc_mma_bf16(tbase + 128 * b + 64, o + ka, dV + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+              }
+            }
+            tc_commit(&s_full[b]);
+            pend[sc_s & 1] = {il_s, first_step ? 1 : 0, last ? 1 : 0, has ? 1 : 0};
+            ++sc_s;
+            first_step = last;
+            if (last) {
+              ++il_s;
+              it_s += gridDim.x;
+            }
+            progress = true;
+          }
+        }
+        if (sc_a < sc_s) {
+          const Pending pa = pend[sc_a & 1];
+          if (mbar_try_wait(pd_full, sc_a & 1) &&
+              (!pa.first || pa.il < 1 || mbar_try_wait(acc_empty, (pa.il - 1) & 1))) {
+            const int ss = sc_a & 1;
+            tc_fence_after();
+            if (pa.has) {
               const uint64_t q = dStMN + ss * kSt16, o = q + kPair16;
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {  // K = 128 query rows
-                const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
+                const uint32_t acc = (acc_started || kk > 0) ? 1u : 0u;
                 tc_mma_bf16(t_dv, o + 128 * kk, dP + 128 * kk, C::kIdescAcc, acc);
                 tc_mma_bf16(t_dk, q + 128 * kk, dDs + 128 * kk, C::kIdescAcc, acc);
               }
-              first = false;
+              acc_started = true;
             }
             tc_commit(pd_free);
             tc_commit(&stage_free[ss]);
-          };
-          if (prev >= 0) {
-            accumulate(prev, prev_has);
-            if (!ok) break;
-          }
-          prev = sc;
-          prev_has = has;
-          ++sc;
-          if (last) {
-            accumulate(prev, prev_has);
-            break;
+            if (pa.last) {
+              tc_commit(acc_full);
+              tc_commit(item_free);
+              acc_started = false;
+            }
+            ++sc_a;
+            progress = true;
           }
         }
-        if (!ok) break;
-        tc_commit(acc_full);
-        tc_commit(item_free);
+        if (progress) {
+          idle_since = clock64();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (clock64() - idle_since > kWaitCycles) {
+          *abort_flag = 1;
+          record_status(g.status, kStatusTimeout);
+          ok = false;
+        }
       }
       tc_commit(drain);
       drain_wait(drain, 0);
@@ -924,8 +1047,10 @@ __global__ void __launch_bounds__(kBwdThreads)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- elementwise
-    const int r = warp * 32 + lane;  // TMEM lane: query row of the pair (S, dP); feature row (dK^T, dV^T)
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;  // TMEM lane: query row of the pair (S, dP); feature row (dK^T, dV^T)
+    const int c0 = 32 * half;           // this thread's 32 key columns
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     int sc = 0, il = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++il) {
@@ -944,30 +1069,31 @@ __global__ void __launch_bounds__(kBwdThreads)
         any = any || Ia >= 0;
         if (!(ok = mbar_wait(&s_full[b], (sc >> 1) & 1, abort_flag, g.status))) break;
         tc_fence_after();
-        float sv[64], dp[64];
-        ld_row64(tbase + lane_addr + 128 * b, sv);
-        ld_row64(tbase + lane_addr + 128 * b + 64, dp);
+        float sv[32], dp[32];
+        tmem_ld32(tbase + lane_addr + 128 * b + c0, sv);
+        tmem_ld32(tbase + lane_addr + 128 * b + 64 + c0, dp);
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[b]);
         const float* nlv = reinterpret_cast<const float*>(stage(s) + 2 * C::kPair);
         const float nl = nlv[r], dl = nlv[128 + r];  // [-lse log2e of both blocks][D of both blocks]
-        uint32_t pk[32], dsk[32];
+        uint32_t pk[16], dsk[16];
 #pragma unroll
-        for (int j = 0; j < 64; j += 2) {
+        for (int j = 0; j < 32; j += 2) {
+          const int jj = c0 + j;  // key within block J
           float e0 = valid ? ex2_approx(fmaf(sv[j], g.sl, nl)) : 0.f;
           float e1 = valid ? ex2_approx(fmaf(sv[j + 1], g.sl, nl)) : 0.f;
           if (diag) {
-            e0 = j <= i ? e0 : 0.f;
-            e1 = j + 1 <= i ? e1 : 0.f;
+            e0 = jj <= i ? e0 : 0.f;
+            e1 = jj + 1 <= i ? e1 : 0.f;
           }
           pk[j / 2] = pack_bf16x2(e0, e1);
           dsk[j / 2] = pack_bf16x2(e0 * (dp[j] - dl), e1 * (dp[j + 1] - dl));
         }
         if (sc >= 1) mbar_wait(pd_free, (sc - 1) & 1, abort_flag, g.status);
-        store_row64(sP, r, pk);
-        store_row64(sDs, r, dsk);
+        store_half_row(sP, r, half, pk);
+        store_half_row(sDs, r, half, dsk);
         fence_async_shared();
         __syncwarp();
         if (lane == 0) mbar_arrive(pd_full);
@@ -980,19 +1106,16 @@ __global__ void __launch_bounds__(kBwdThreads)
       if (r < D) {  // warp-uniform
         const size_t pj = (static_cast<size_t>(bh) * g.M + J) * D + r;
         const float kb = dkbar[pj] * (1.0f / 64.0f), vs = dvsum[pj];
-        const size_t o = (static_cast<size_t>(bh) * g.N + 64 * J) * D + r;
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          float a[32], c[32];
-          tmem_ld32(t_dk + lane_addr + 32 * h, a);
-          tmem_ld32(t_dv + lane_addr + 32 * h, c);
-          tc_wait_ld();
+        const size_t o = (static_cast<size_t>(bh) * g.N + 64 * J + c0) * D + r;
+        float a[32], c[32];
+        tmem_ld32(t_dk + lane_addr + c0, a);
+        tmem_ld32(t_dv + lane_addr + c0, c);
+        tc_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const size_t oj = o + static_cast<size_t>(32 * h + j) * D;
-            dk[oj] = __float2bfloat16_rn((any ? g.tau * a[j] : 0.f) + kb);
-            dv[oj] = __float2bfloat16_rn((any ? c[j] : 0.f) + vs);
-          }
+        for (int j = 0; j < 32; ++j) {
+          const size_t oj = o + static_cast<size_t>(j) * D;
+          dk[oj] = __float2bfloat16_rn((any ? g.tau * a[j] : 0.f) + kb);
+          dv[oj] = __float2bfloat16_rn((any ? c[j] : 0.f) + vs);
         }
       }
       tc_fence_before();
@@ -1002,7 +1125,7 @@ __global__ void __launch_bounds__(kBwdThreads)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }

@@ -560,3 +560,18 @@ def test_full_dit_video_wide_logits():
     qbar, kbar, vsum = check_pool(g, q, k, v)
     check_routing(g, O.block_scores(qbar, kbar), "topk", 0.15, False)
     _check_wide(g, q, k, v, sample_units(w["B"], w["H"], w["N"] // 64, 40, seed=10, g=g))
+
+
+# ------------------------------------------------------------------ FlashPrefill's fused scoring (reading r18)
+@pytest.mark.parametrize("mode,param", [("topk", 0.15), ("thresh", 0.5)])
+def test_routing_equals_token_pooled_scores(mode, param):
+    # FlashPrefill summary, 2.a: the token queries scored against the pooled
+    # key of each block, then pooled over the query block.  With mean pooling
+    # that is q-bar . k-bar / sqrt(d), which the tensor-core scorer computes;
+    # the GPU's lists must equal the lists the oracle's token-level scores give
+    q, k, v = make_qkv(1, 2, 256 * 64, 128, "clustered", seed=53)
+    g = run_gpu(q, k, v, mode, param)
+    assert g["status"] == psa.PSA_OK
+    _, kbar, _ = O.pool(f64(q), f64(k), f64(v))
+    s_tok = O.token_pooled_block_scores(f64(q), kbar)
+    check_routing(g, s_tok, mode, param, False)
