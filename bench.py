@@ -186,28 +186,28 @@ class Step:
         self.launches = launches_per_step(B, H, self.M, self.mode, dense, hyd)
 
     def run(self, ev=None, io=None, stream=None):
-        """pool -> route -> [statistic ->] attention; ``ev`` = 5 events to split
-        the kernels (pool | route | first-order statistic | attention);
+        """pool -> route -> [statistic ->] attention; ``ev`` = 5 events (or
+        None entries) recorded before the pool, after it, after the routing,
+        after the first-order statistic and after the attention call;
         ``io`` = (q, k, v, out) device tensors (default: the step's own) and
         ``stream`` the stream to issue on (default: the current one)."""
         q, k, v, out = io if io is not None else (self.q, self.k, self.v, self.out)
         s = stream if stream is not None else self.stream
+
+        def mark(i):
+            if ev is not None and ev[i] is not None:
+                ev[i].record(s)
+
         if self.dense:
             # the dense baseline: one call (it pools the keys for its stabiliser itself)
-            if ev:
-                ev[0].record(s)
-                ev[1].record(s)
-                ev[2].record(s)
-                ev[3].record(s)
+            for i in range(4):
+                mark(i)
             psa.psa_dense(q, k, v, self.causal, ws=self.ws, out=out, stream=s)
-            if ev:
-                ev[4].record(s)
+            mark(4)
             return
-        if ev:
-            ev[0].record(s)
+        mark(0)
         psa.psa_pool(q, k, v, out=self.stats, stream=s)
-        if ev:
-            ev[1].record(s)
+        mark(1)
         qbar, kbar, vsum = self.stats
         if self.mode == "topk":
             psa.psa_route_topk(qbar, kbar, self.param, self.causal, out=self.csr, ws=self.ws, stream=s)
@@ -217,20 +217,17 @@ class Step:
         else:
             psa.psa_route_thresh(qbar, kbar, self.param, self.causal, self.keep_first, ws=self.ws,
                                  out=self.csr, stream=s)
-        if ev:
-            ev[2].record(s)
+        mark(2)
         if self.hyd:
             psa.psa_hyd_stat(k, v, kbar, vsum, ws=self.ws, out=self.hstat, stream=s)
-        if ev:
-            ev[3].record(s)
+        mark(3)
         if self.hyd:
             psa.psa_attn_hyd(q, k, v, kbar, vsum, self.hstat, self.csr[0], self.csr[1], self.causal, ws=self.ws,
                              out=out, row_max=self.csr[3], stream=s)
         else:
             psa.psa_attn(q, k, v, kbar, vsum, self.csr[0], self.csr[1], self.causal, ws=self.ws,
                          out=out, row_max=self.csr[3], stream=s)
-        if ev:
-            ev[4].record(s)
+        mark(4)
 
     def e2e_ms(self, nsteps):
         """Milliseconds per step with host buffers in and the host result out,
@@ -278,21 +275,22 @@ class Step:
 
 
 def launches_per_step(B: int, H: int, M: int, mode: str, dense: bool, hyd: bool = False) -> int:
-    """Kernels of ours one step launches: psa_dense = 4 (key pooling,
-    attention, rerun of flagged blocks, exact fixup); otherwise pool 1, route
-    = one split of both operands plus, per batch of heads, one score and one
+    """Kernels of ours one step launches.  Every call that takes a workspace
+    starts with one launch that zeroes its header.  psa_dense = 5 (header,
+    key pooling, attention, rerun of flagged blocks, exact fixup); otherwise
+    pool 1, route = header plus, per batch of heads, one score and one
     selection launch (the library batches as many heads as fit 256 MB of
-    scores), plus scan and compaction for the threshold routers, and attention
-    4 (bf16 statistics, attention, rerun of flagged blocks, exact fixup); the
-    first-order mode adds the statistic (2: partial sums and their reduction)
-    and the correction (1)."""
+    scores), plus scan and compaction for the threshold routers, and
+    attention 5 (header, bf16 statistics, attention, rerun of flagged blocks,
+    exact fixup); the first-order mode adds the statistic call (3: header,
+    partial sums and their reduction) and the correction (1)."""
     if dense:
-        return 4
+        return 5
     Mp = -(-M // 128) * 128
     per_batch = max(1, min(B * H, (256 << 20) // (M * Mp * 4)))
     nb = -(-(B * H) // per_batch)
     route = 1 + 2 * nb + (0 if mode == "topk" else 2)
-    return 1 + route + 4 + (3 if hyd else 0)
+    return 1 + route + 5 + (4 if hyd else 0)
 
 
 def _flush(buf):
@@ -377,20 +375,41 @@ def gpu_arm(args):
 
     clocks = ClockSampler(local)
     clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # the step: one event on each side, so nothing but the library's own
+    # launches sits between its calls (each call's kernels are chained
+    # launches that start while the previous kernel drains)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     _barrier(world)
     torch.cuda.synchronize()
     for i in range(args.steps):
-        st.run(evs[i])
+        evs[i][0].record(st.stream)
+        st.run()
+        evs[i][1].record(st.stream)
         _flush(flush)
     torch.cuda.synchronize()
+    # the per-call split: the same steps twice more, with events between
+    # some calls (an event between two calls serialises them, so these times
+    # feed the kernel split and the roofline, not the step time): once with
+    # pool + routing as one chained pass, the statistic and the attention
+    # call each between events; once with the pool alone between events
+    def timed(marks):
+        out = []
+        for _ in range(args.steps):
+            ev = [torch.cuda.Event(enable_timing=True) if m else None for m in marks]
+            st.run(ev)
+            _flush(flush)
+            out.append(ev)
+        torch.cuda.synchronize()
+        return out
+    split = timed((1, 0, 1, 1, 1))
+    pool_only = timed((1, 1, 0, 0, 0))
     _barrier(world)
     clk = clocks.stop()
-    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
-    pool_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    route_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    stat_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    attn_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    pool_ms = [e[0].elapsed_time(e[1]) for e in pool_only]
+    pool_route_ms = [e[0].elapsed_time(e[2]) for e in split]
+    stat_ms = [e[2].elapsed_time(e[3]) for e in split]
+    attn_ms = [e[3].elapsed_time(e[4]) for e in split]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
 
@@ -405,7 +424,8 @@ def gpu_arm(args):
     attn_avg = statistics.mean(attn_ms)
     stat_avg = statistics.mean(stat_ms)
     pool_avg = statistics.mean(pool_ms)
-    route_avg = statistics.mean(route_ms)
+    pool_route_avg = statistics.mean(pool_route_ms)
+    route_avg = pool_route_avg - pool_avg  # what the routing adds to the chained pass
     achieved = ex_flops / (attn_avg * 1e-3) / 1e12
     tc_peak = peaks["bf16_tflops"]
     line = {
@@ -443,10 +463,12 @@ def gpu_arm(args):
                     "pool_gbs": None if st.dense else round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3) / 1e9, 1),
                     "pool_hbm_frac": None if st.dense else round(pool_bytes(st.B, st.H, st.N, st.d) / (pool_avg * 1e-3)
                                                                  / 1e9 / peaks["hbm_gbs"], 4),
-                    # pool and route as one pass over the pooled inputs' HBM bytes (the
-                    # routing itself reads only the pooled statistics)
+                    # pool and route as one chained pass (timed between two events)
+                    # over the pooled inputs' HBM bytes (the routing itself reads
+                    # only the pooled statistics)
+                    "pool_route_ms": None if st.dense else round(pool_route_avg, 4),
                     "pool_route_hbm_frac": None if st.dense else round(
-                        pool_bytes(st.B, st.H, st.N, st.d) / ((pool_avg + route_avg) * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                        pool_bytes(st.B, st.H, st.N, st.d) / (pool_route_avg * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                     "attn_executed_tflops": round(achieved, 2),
                     "attn_effective_tflops": round(de_flops / (attn_avg * 1e-3) / 1e12, 2)},
         "flops": {"dense_equivalent": de_flops, "executed": ex_flops, "mma_issued": is_flops,
@@ -544,7 +566,8 @@ def bwd_arm(args):
                      "peak_source": peaks["source"] + " bf16 burst"},
         "flops": {"dense_equivalent": de, "executed": ex},
         "device_status": status,
-        "gpu_launches": 7 * args.steps,  # bf16 statistics, delta, bitmaps, pseudo + its reduction, dq, dk/dv
+        # header, bf16 statistics, delta, bitmaps, pseudo + its reduction, dq, dk/dv
+        "gpu_launches": 8 * args.steps,
         "clocks": clk,
     }
     if rank == 0:

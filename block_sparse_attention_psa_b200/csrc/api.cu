@@ -177,7 +177,7 @@ int route_thresh_common(const float* qbar, const float* kbar, int B, int H, int 
   const long long cap = capacity > static_cast<size_t>(INT_MAX) ? INT_MAX : static_cast<long long>(capacity);
   char* ws = static_cast<char*>(workspace);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
+  if (psa::launch_zero_header(ws, st) != cudaSuccess) return PSA_ERR_CUDA;
   return cuda_status(psa::launch_route_thresh(qbar, kbar, static_cast<int>(bh), M, d, a_mul, a_add, causal,
                                               keep_first, row_ptr, col_idx, cap, nnz_out,
                                               reinterpret_cast<int*>(ws + L.row_count),
@@ -206,7 +206,7 @@ int attn_common(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, c
   if ((s = check_device({q, out, workspace})) != PSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
+  cudaError_t e = psa::launch_zero_header(ws, st);
   if (e != cudaSuccess) return PSA_ERR_CUDA;
   uint16_t* kb16 = reinterpret_cast<uint16_t*>(ws + L.kbar_bf16);
   uint16_t* vb16 = reinterpret_cast<uint16_t*>(ws + L.vsum_bf16);
@@ -315,7 +315,7 @@ int psa_route_topk(const float* qbar, const float* kbar, int B, int H, int M, in
   if ((s = check_device({qbar, row_ptr, workspace})) != PSA_OK) return s;
   char* ws = static_cast<char*>(workspace);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
+  if (psa::launch_zero_header(ws, st) != cudaSuccess) return PSA_ERR_CUDA;
   return cuda_status(psa::launch_route_topk(qbar, kbar, static_cast<int>(bh), M, d, static_cast<int>(k0),
                                             causal, row_ptr, col_idx, total, nnz_out, row_max,
                                             route_scratch(ws, L), st));
@@ -377,7 +377,7 @@ int psa_attn_bwd(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, 
   if ((s = check_device({q, dout, dq, workspace})) != PSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
+  if (psa::launch_zero_header(ws, st) != cudaSuccess) return PSA_ERR_CUDA;
   uint16_t* kb16 = reinterpret_cast<uint16_t*>(ws + L.kbar_bf16);
   uint16_t* vb16 = reinterpret_cast<uint16_t*>(ws + L.vsum_bf16);
   if (psa::launch_stats_to_bf16(kbar, vsum, bh * M * d, kb16, vb16, st) != cudaSuccess) return PSA_ERR_CUDA;
@@ -429,7 +429,7 @@ int psa_hyd_stat(const psa_bf16_t* k, const psa_bf16_t* v, const float* kbar, co
   if ((s = check_device({k, hstat, workspace})) != PSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
+  if (psa::launch_zero_header(ws, st) != cudaSuccess) return PSA_ERR_CUDA;
   return cuda_status(psa::launch_hyd_stat(k, v, kbar, vsum, static_cast<int>(bh), N, d,
                                           reinterpret_cast<float*>(ws + L.hyd_partial), hstat,
                                           reinterpret_cast<int*>(ws), st));
@@ -451,7 +451,7 @@ int psa_dense(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, int
   if ((s = check_device({q, out, workspace})) != PSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
+  cudaError_t e = psa::launch_zero_header(ws, st);
   if (e != cudaSuccess) return PSA_ERR_CUDA;
   uint16_t* kb16 = reinterpret_cast<uint16_t*>(ws + L.kbar_bf16);
   e = psa::launch_pool_keys_bf16(k, static_cast<int>(bh), M, d, kb16, st);

@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // the units of this launch: every (head, query block), or in rerun mode the
   // first pass's list (unit ids from it)
-  const int units = FIX ? *p.fix_src_count : p.units;
+  int units = p.units;  // rerun mode: read after the wait for the first pass
   auto uid = [&](int u) { return FIX ? __ldg(p.fix_src_list + u) : u; };
   // Dynamic unit scheduler.  A CTA's first unit is blockIdx.x; each later one
   // is the next ticket of the launch's counter (after the grid's first
@@ -388,6 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  grid_dep_launch();
+  grid_dep_wait();
+  if (FIX) units = *p.fix_src_count;
 
   if (warp < 4) {
   reg_dealloc<kRegsProducer>();
@@ -903,6 +906,8 @@ __global__ void __launch_bounds__(64) fixup_kernel(const __nv_bfloat16* __restri
   float(*qs)[D + 1] = reinterpret_cast<float(*)[D + 1]>(fx_sm);
   float(*num)[D + 1] = reinterpret_cast<float(*)[D + 1]>(fx_sm + 64 * (D + 1));
   uint32_t* listed = reinterpret_cast<uint32_t*>(fx_sm + 128 * (D + 1));
+  grid_dep_launch();
+  grid_dep_wait();
   const int n = *p.fixup_count;
   const int i = threadIdx.x;
   const float tau = p.scale_log2 * kLn2;  // 1 / sqrt(d)
@@ -1039,8 +1044,9 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   if ((e = prepare_attn_kernel<D, HYD, true>(kSmem)) != cudaSuccess) return e;
   const int sms = device_sm_count();
   const int grid = p.units < sms ? p.units : sms;
-  attn_kernel<D, HYD, false><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, mkb, mvb, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_chained(attn_kernel<D, HYD, false>, dim3(grid), dim3(kThreads), kSmem, st, mq, mk, mv, mkb, mvb,
+                         p)) != cudaSuccess)
+    return e;
   // the rerun: the first pass's list in, a second list out
   Params r = p;
   r.stall = 0;
@@ -1051,8 +1057,9 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   r.fixup_count = a.fixup_count2;
   r.fixup_list = a.fixup_list2;
   r.sched = a.sched + 1;
-  attn_kernel<D, HYD, true><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, mkb, mvb, r);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_chained(attn_kernel<D, HYD, true>, dim3(grid), dim3(kThreads), kSmem, st, mq, mk, mv, mkb, mvb,
+                         r)) != cudaSuccess)
+    return e;
   // exact recomputation of what the rerun still flags
   Params f = p;
   f.fixup_count = a.fixup_count2;
@@ -1061,10 +1068,9 @@ cudaError_t launch_d(const AttnLaunch& a, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(fixup_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(fx_smem))) != cudaSuccess)
     return e;
-  fixup_kernel<D><<<64, 64, fx_smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(a.q),
-                                           reinterpret_cast<const __nv_bfloat16*>(a.k),
-                                           reinterpret_cast<const __nv_bfloat16*>(a.v), f, a.N);
-  return cudaGetLastError();
+  return launch_chained(fixup_kernel<D>, dim3(64), dim3(64), fx_smem, st, reinterpret_cast<const __nv_bfloat16*>(a.q),
+                        reinterpret_cast<const __nv_bfloat16*>(a.k), reinterpret_cast<const __nv_bfloat16*>(a.v), f,
+                        a.N);
 }
 
 }  // namespace

@@ -5,10 +5,31 @@
 #include <cstddef>
 #include <cstdint>
 #include <initializer_list>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace psa {
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream is still running (after that one
+// calls grid_dep_launch() in every CTA); the kernel itself calls
+// grid_dep_wait() before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                           Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 constexpr int kBlock = 64;        // tokens per block (the only supported size)
 constexpr int kMaxBlocks = 16384; // M limit (bitmaps and score rows on chip)
@@ -62,6 +83,8 @@ cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         float* qbar, float* kbar, float* vsum, cudaStream_t st);
 cudaError_t launch_pool_keys_bf16(const uint16_t* k, int BH, int M, int d, uint16_t* kbar_bf16,
                                   cudaStream_t st);
+// zero the 256-byte header of a workspace (a chained launch, in place of a memset)
+cudaError_t launch_zero_header(void* workspace, cudaStream_t st);
 cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long n, uint16_t* kbar_bf16,
                                  uint16_t* vsum_bf16, cudaStream_t st);
 

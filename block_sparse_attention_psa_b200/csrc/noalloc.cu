@@ -129,7 +129,7 @@ int psa_attn_noalloc(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t*
   const size_t off_lse2 = off_fix2 + align256(static_cast<size_t>(bh * M) * 4);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the status word and the fixup counter must start at zero on every call
-  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return PSA_ERR_CUDA;
+  if (psa::launch_zero_header(ws, st) != cudaSuccess) return PSA_ERR_CUDA;
   uint16_t* kb16 = reinterpret_cast<uint16_t*>(ws + off_kb);
   uint16_t* vs16 = reinterpret_cast<uint16_t*>(ws + off_vs);
   if (psa::launch_stats_to_bf16(kbar, vsum, bh * M * d, kb16, vs16, st) != cudaSuccess) return PSA_ERR_CUDA;

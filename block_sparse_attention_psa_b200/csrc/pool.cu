@@ -47,6 +47,8 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ q, 
   const int g = threadIdx.x / kChunks;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int items = nblk * NT;
+  grid_dep_launch();
+  grid_dep_wait();
 
   for (int it = blockIdx.x; it < items; it += gridDim.x) {
     const int blk = it / NT, t = it - blk * NT;
@@ -87,8 +89,17 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ q, 
   }
 }
 
+// Zero the 256-byte header of a call's workspace (status word, counters).
+__global__ void zero_header_kernel(int4* __restrict__ header) {
+  grid_dep_launch();
+  grid_dep_wait();
+  if (threadIdx.x < 16) header[threadIdx.x] = make_int4(0, 0, 0, 0);
+}
+
 __global__ void stats_to_bf16_kernel(const float4* __restrict__ kbar, const float4* __restrict__ vsum,
                                      long long n4, uint2* __restrict__ kb, uint2* __restrict__ vb) {
+  grid_dep_launch();
+  grid_dep_wait();
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const float4 a = kbar[i];
@@ -114,11 +125,9 @@ cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   auto* Q = reinterpret_cast<const uint4*>(q);
   auto* K = reinterpret_cast<const uint4*>(k);
   auto* V = reinterpret_cast<const uint4*>(v);
-  if (d == 128)
-    pool_kernel<128, 3><<<grid, 256, 0, st>>>(Q, K, V, nblk, qbar, kbar, vsum, nullptr);
-  else
-    pool_kernel<64, 3><<<grid, 256, 0, st>>>(Q, K, V, nblk, qbar, kbar, vsum, nullptr);
-  return cudaGetLastError();
+  uint16_t* none = nullptr;
+  if (d == 128) return launch_chained(pool_kernel<128, 3>, grid, dim3(256), 0, st, Q, K, V, nblk, qbar, kbar, vsum, none);
+  return launch_chained(pool_kernel<64, 3>, grid, dim3(256), 0, st, Q, K, V, nblk, qbar, kbar, vsum, none);
 }
 
 cudaError_t launch_pool_keys_bf16(const uint16_t* k, int BH, int M, int d, uint16_t* kbar_bf16,
@@ -126,11 +135,13 @@ cudaError_t launch_pool_keys_bf16(const uint16_t* k, int BH, int M, int d, uint1
   const int nblk = BH * M;
   const dim3 grid(pool_grid(nblk));
   auto* K = reinterpret_cast<const uint4*>(k);
+  const uint4* none = nullptr;
+  float* nonef = nullptr;
   if (d == 128)
-    pool_kernel<128, 1><<<grid, 256, 0, st>>>(nullptr, K, nullptr, nblk, nullptr, nullptr, nullptr, kbar_bf16);
-  else
-    pool_kernel<64, 1><<<grid, 256, 0, st>>>(nullptr, K, nullptr, nblk, nullptr, nullptr, nullptr, kbar_bf16);
-  return cudaGetLastError();
+    return launch_chained(pool_kernel<128, 1>, grid, dim3(256), 0, st, none, K, none, nblk, nonef, nonef, nonef,
+                          kbar_bf16);
+  return launch_chained(pool_kernel<64, 1>, grid, dim3(256), 0, st, none, K, none, nblk, nonef, nonef, nonef,
+                        kbar_bf16);
 }
 
 cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long n, uint16_t* kbar_bf16,
@@ -140,10 +151,13 @@ cudaError_t launch_stats_to_bf16(const float* kbar, const float* vsum, long long
   const long long cap = device_sm_count() * 16LL;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  stats_to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      reinterpret_cast<const float4*>(kbar), reinterpret_cast<const float4*>(vsum), n4,
-      reinterpret_cast<uint2*>(kbar_bf16), reinterpret_cast<uint2*>(vsum_bf16));
-  return cudaGetLastError();
+  return launch_chained(stats_to_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+                        reinterpret_cast<const float4*>(kbar), reinterpret_cast<const float4*>(vsum), n4,
+                        reinterpret_cast<uint2*>(kbar_bf16), reinterpret_cast<uint2*>(vsum_bf16));
+}
+
+cudaError_t launch_zero_header(void* workspace, cudaStream_t st) {
+  return launch_chained(zero_header_kernel, dim3(1), dim3(32), 0, st, static_cast<int4*>(workspace));
 }
 
 }  // namespace psa

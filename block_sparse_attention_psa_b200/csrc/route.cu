@@ -118,6 +118,8 @@ __global__ void __launch_bounds__(256, 4) route_topk_kernel(const float* __restr
                                                          long long total, int* __restrict__ nnz_out,
                                                          float* __restrict__ row_max) {
   extern __shared__ float ss[];  // [R][Mp] score rows, then [R][256] histograms
+  grid_dep_launch();
+  grid_dep_wait();
   const int hl = blockIdx.y, bh = bh0 + hl;
   const int I0 = blockIdx.x * R;
   const int rows = min(R, M - I0);
@@ -229,6 +231,8 @@ __global__ void __launch_bounds__(256, 4) route_thresh_kernel(const float* __res
                                                            uint32_t* __restrict__ row_bits,
                                                            float* __restrict__ row_max) {
   extern __shared__ float ss[];  // [R][Mp] score rows
+  grid_dep_launch();
+  grid_dep_wait();
   const int hl = blockIdx.y, bh = bh0 + hl;
   const int I0 = blockIdx.x * R;
   const int rows = min(R, M - I0);
@@ -267,6 +271,8 @@ __global__ void __launch_bounds__(1024) scan_rows_kernel(const int* __restrict__
                                                          long long capacity, int* __restrict__ row_ptr,
                                                          int* __restrict__ nnz_out) {
   constexpr int kItems = 8;
+  grid_dep_launch();
+  grid_dep_wait();
   __shared__ long long warp_tot[32];
   __shared__ long long carry_s;
   const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
@@ -322,6 +328,8 @@ __global__ void __launch_bounds__(1024) scan_rows_kernel(const int* __restrict__
 __global__ void __launch_bounds__(256) compact_rows_kernel(const uint32_t* __restrict__ row_bits,
                                                            const int* __restrict__ row_ptr, long long nrows,
                                                            int M, int causal, int* __restrict__ col_idx) {
+  grid_dep_launch();
+  grid_dep_wait();
   const int lane = threadIdx.x % 32;
   const long long row = blockIdx.x * 8LL + threadIdx.x / 32;
   if (row >= nrows) return;
@@ -386,8 +394,8 @@ cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int 
 #define PSA_TOPK(RR)                                                                                         \
   case RR:                                                                                                   \
     if ((e = set_smem(route_topk_kernel<RR>, smem)) != cudaSuccess) return e;                                \
-    route_topk_kernel<RR><<<grid, 256, smem, st>>>(w.scores, Mp, h0, BH, M, k0, causal, row_ptr, col_idx,    \
-                                                   total, nnz_out, row_max);                                 \
+    e = launch_chained(route_topk_kernel<RR>, grid, dim3(256), smem, st, w.scores, Mp, h0, BH, M, k0, causal, \
+                       row_ptr, col_idx, total, nnz_out, row_max);                                           \
     break;
     switch (R) {
       PSA_TOPK(8)
@@ -398,7 +406,7 @@ cudaError_t launch_route_topk(const float* qbar, const float* kbar, int BH, int 
         return cudaErrorInvalidValue;
     }
 #undef PSA_TOPK
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
 }
@@ -420,8 +428,8 @@ cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, in
 #define PSA_THRESH(RR)                                                                                       \
   case RR:                                                                                                   \
     if ((e = set_smem(route_thresh_kernel<RR>, smem)) != cudaSuccess) return e;                              \
-    route_thresh_kernel<RR><<<grid, 256, smem, st>>>(w.scores, Mp, h0, M, a_mul, a_add, causal, keep_first,  \
-                                                     row_count, row_bits, row_max);                          \
+    e = launch_chained(route_thresh_kernel<RR>, grid, dim3(256), smem, st, w.scores, Mp, h0, M, a_mul, a_add, \
+                       causal, keep_first, row_count, row_bits, row_max);                                    \
     break;
     switch (R) {
       PSA_THRESH(8)
@@ -432,14 +440,15 @@ cudaError_t launch_route_thresh(const float* qbar, const float* kbar, int BH, in
         return cudaErrorInvalidValue;
     }
 #undef PSA_THRESH
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (e != cudaSuccess) return e;
   }
   const long long nrows = static_cast<long long>(BH) * M;
-  scan_rows_kernel<<<1, 1024, 0, st>>>(row_count, nrows, capacity, row_ptr, nnz_out);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  compact_rows_kernel<<<static_cast<unsigned>((nrows + 7) / 8), 256, 0, st>>>(row_bits, row_ptr, nrows, M,
-                                                                               causal, col_idx);
-  return cudaGetLastError();
+  if ((e = launch_chained(scan_rows_kernel, dim3(1), dim3(1024), 0, st, static_cast<const int*>(row_count), nrows,
+                         capacity, row_ptr, nnz_out)) != cudaSuccess)
+    return e;
+  return launch_chained(compact_rows_kernel, dim3(static_cast<unsigned>((nrows + 7) / 8)), dim3(256), 0, st,
+                        static_cast<const uint32_t*>(row_bits), static_cast<const int*>(row_ptr), nrows, M, causal,
+                        col_idx);
 }
 
 }  // namespace psa

@@ -50,6 +50,8 @@ constexpr uint32_t kScoreIdesc = idesc_bf16_f32(128, 128, 0, 0);
 __global__ void __launch_bounds__(256) split3_kernel(const float4* __restrict__ x0, const float4* __restrict__ x1,
                                                      long long n4, uint2* __restrict__ out0,
                                                      uint2* __restrict__ out1) {
+  grid_dep_launch();
+  grid_dep_wait();
   for (long long t = blockIdx.x * 256LL + threadIdx.x; t < 2 * n4; t += static_cast<long long>(gridDim.x) * 256) {
     const bool second = t >= n4;
     const long long i = second ? t - n4 : t;
@@ -81,7 +83,7 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
                                                        float* __restrict__ scores, int* status) {
   constexpr int kChunks = D / 64;
   const int tj = blockIdx.x, ti = blockIdx.y, hl = blockIdx.z;
-  if (causal && tj > ti) return;  // every J of the tile is above every I
+  if (causal && tj > ti) return;  // every J of the tile is above every I (an exit counts as the trigger)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                  // query parts of one chunk [3][128 x 64]
@@ -111,6 +113,8 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  grid_dep_launch();
+  grid_dep_wait();
 
   const int I0 = ti * kTile, J0 = tj * kTile;
   const int rowQ = (bh0 + hl) * M + I0, rowK = (bh0 + hl) * M + J0;
@@ -190,8 +194,8 @@ cudaError_t launch_score_tiles(const CUtensorMap& mq, const CUtensorMap& mk, int
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
   if (e != cudaSuccess) return e;
   const int nt = (M + kTile - 1) / kTile;
-  score_tc_kernel<D><<<dim3(nt, nt, nh), 128, kScoreSmem, st>>>(mq, mk, M, Mp, bh0, causal, tau, scores, status);
-  return cudaGetLastError();
+  return launch_chained(score_tc_kernel<D>, dim3(nt, nt, nh), dim3(128), kScoreSmem, st, mq, mk, M, Mp, bh0, causal,
+                        tau, scores, status);
 }
 
 }  // namespace
@@ -204,9 +208,9 @@ cudaError_t launch_split3(const float* x0, const float* x1, long long n, uint16_
   if (n4 == 0) return cudaSuccess;
   const long long want = (2 * n4 + 255) / 256;
   const int grid = static_cast<int>(want < 148LL * 16 ? want : 148LL * 16);
-  split3_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(x0), reinterpret_cast<const float4*>(x1), n4,
-                                      reinterpret_cast<uint2*>(out0), reinterpret_cast<uint2*>(out1));
-  return cudaGetLastError();
+  return launch_chained(split3_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const float4*>(x0),
+                        reinterpret_cast<const float4*>(x1), n4, reinterpret_cast<uint2*>(out0),
+                        reinterpret_cast<uint2*>(out1));
 }
 
 cudaError_t ScorePlan::init(const uint16_t* qs, const uint16_t* ks, int BH_, int M_, int d_) {

@@ -94,6 +94,21 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ---------------------------------------------------------------- launch chaining
+// Programmatic dependent launch.  A kernel of this library launched with the
+// programmatic-serialization attribute may start while the kernel before it
+// in the stream is still running; it touches no global memory before
+// grid_dep_wait(), which returns once every grid it depends on has completed
+// and its writes are visible (at once for a plain launch).  Because every
+// kernel of a chain waits this way, the wait also covers the grids further
+// back.  grid_dep_launch() lets the next launch of the stream be scheduled
+// as soon as every CTA of this grid has called it (or exited); a kernel that
+// holds tensor memory calls it only after its allocation has succeeded, so a
+// dependent CTA on the same SM can never hold columns this CTA still waits
+// for.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -60,15 +60,16 @@ def test_dense_flops_formula():
 
 
 def test_launches_per_step_matches_the_launch_lists():
-    # launch lists of one step (pool, split3, score_tc, selection, stats_to_bf16,
-    # attention, its rerun of flagged blocks, fixup; + scan and compaction for
-    # the threshold routers)
-    assert bench.launches_per_step(1, 12, 512, "topk", False) == 8
-    assert bench.launches_per_step(1, 12, 512, "thresh", False) == 10
-    assert bench.launches_per_step(1, 8, 2048, "thresh", False) == 10      # 8 x 16 MB of scores: one batch
-    assert bench.launches_per_step(1, 1, 16384, "topk", False) == 8
-    assert bench.launches_per_step(1, 2, 16384, "topk", False) == 10       # 1 GB per head: two batches
-    assert bench.launches_per_step(1, 12, 512, "topk", True) == 4
+    # launch lists of one step (pool; route: header, score_tc, selection; attention:
+    # header, stats_to_bf16, the sweep, its rerun of flagged blocks, fixup; + scan and
+    # compaction for the threshold routers)
+    assert bench.launches_per_step(1, 12, 512, "topk", False) == 9
+    assert bench.launches_per_step(1, 12, 512, "thresh", False) == 11
+    assert bench.launches_per_step(1, 8, 2048, "thresh", False) == 11      # 8 x 16 MB of scores: one batch
+    assert bench.launches_per_step(1, 1, 16384, "topk", False) == 9
+    assert bench.launches_per_step(1, 2, 16384, "topk", False) == 11       # 1 GB per head: two batches
+    assert bench.launches_per_step(1, 12, 512, "topk", True) == 5
+    assert bench.launches_per_step(1, 12, 512, "topk", False, hyd=True) == 13
 
 
 def test_reference_arm_prints_its_line_on_the_host():
