@@ -73,8 +73,8 @@ def executed_flops(row_ptr, col_idx, B, H, M, d, causal):
 
 def issued_flops(row_ptr, B, H, M, d, causal, dense=False):
     """FLOPs the attention kernel's MMAs issue (host, from the block lists):
-    per tile S^T = K Q^T (128 x 64 x d) and O^T += V^T P^T (128 x 64 x 128,
-    M = 128 rows even when d = 64).  A unit takes ceil(listed / 2) exact tiles
+    per tile S^T = K Q^T (128 x 64 x d) and O^T += V^T P^T (d x 64 x 128: an
+    M = d product).  A unit takes ceil(listed / 2) exact tiles
     and, when some candidate is unlisted, ceil(pooled candidates / 128) pooled
     tiles (at least one tile in all)."""
     rp = row_ptr.astype(np.int64)
@@ -85,7 +85,7 @@ def issued_flops(row_ptr, B, H, M, d, causal, dense=False):
     n_a2 = np.where((~np.bool_(dense)) & (pcand > 0) & (nsel < cand), (pcand + 127) // 128, 0)
     n_e = (nsel + 1) // 2
     tiles = np.maximum(n_a2 + n_e, 1)
-    return float(tiles.sum()) * (2.0 * 128 * 64 * d + 2.0 * 128 * 64 * 128)
+    return float(tiles.sum()) * (2.0 * 128 * 64 * d + 2.0 * d * 64 * 128)
 
 
 def pool_bytes(B, H, N, d):

@@ -83,9 +83,12 @@ struct Cfg {
   static_assert(kOffOnes % 16 == 0, "no-swizzle operand alignment");
   static_assert(kSmemBytesHyd <= 232448, "shared memory of one CTA");
   // kind::f16, bf16 x bf16 -> f32.  GEMM1: M=128 keys, N=64 queries, both
-  // K-major.  GEMM2: M=128 (feature rows), N=64 queries, both MN-major.
+  // K-major.  GEMM2: M=d (feature rows), N=64 queries, both MN-major.  An
+  // M = 64 product takes as many cycles as an M = 128 one but reads half the
+  // A operand from shared memory, the resource the products compete for.  Its
+  // accumulator row m sits in TMEM lane 32 (m / 16) + m % 16.
   static constexpr uint32_t kIdesc1 = idesc_bf16_f32(128, 64, 0, 0);
-  static constexpr uint32_t kIdesc2 = idesc_bf16_f32(128, 64, 1, 1);
+  static constexpr uint32_t kIdesc2 = idesc_bf16_f32(D, 64, 1, 1);
   // hyd mode: R[128 x 64 queries] += ONES[128 x 128 keys] . P^T (A K-major)
   static constexpr uint32_t kIdescOnes = idesc_bf16_f32(128, 64, 0, 1);
 };
@@ -524,8 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // O^T[unit parity] += V_tile^T . P^T for every A2 / E tile, in order.
     if (lane == 0) {
       const uint64_t dV0 = sdesc_sw128(smem_u32(sV), D == 128 ? 16384 : 0, 1024);
-      // V viewed MN-major: feature atoms 16 KB apart (d = 64: the second
-      // atom repeats the first and its output rows are never read)
+      // V viewed MN-major: feature atoms 16 KB apart (d = 64: one atom)
       const uint64_t dP0 = sdesc_sw128(smem_u32(sP), 16, 1024);
       // all-ones A operand (hyd mode): 16 core matrices of 8 rows along M
       // (256 B apart), 2 along K (128 B apart) -- 4 KB, every byte 1.0
@@ -827,16 +829,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ob = ul & 1;
         mbar_wait(&o_full[ob], (ul >> 1) & 1, abort_flag, p.status);
         tc_fence_after();
-        if (trow < D) {  // warp-uniform
+        // feature row of O^T in this thread's TMEM lane (d = 64: the M = 64
+        // layout, 16 rows per lane quarter)
+        {
+          const int frow = D == 128 ? trow : wq * 16 + (lane & 15);
           __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sOut);
 #pragma unroll 1
           for (int h = 0; h < 2; ++h) {
             float ov[32];
-            tmem_ld32(tbase + lane_addr + 128 + 64 * ob + 32 * h, ov);
+            tmem_ld32(tbase + lane_addr + 128 + 64 * ob + 32 * h, ov);  // every lane (aligned)
             tc_wait_ld();
+            if (D == 128 || lane < 16) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q)
-              st[(32 * h + q) * D + trow] = __float2bfloat16_rn(ov[q] * invl[32 * h + q]);
+              for (int q = 0; q < 32; ++q)
+                st[(32 * h + q) * D + frow] = __float2bfloat16_rn(ov[q] * invl[32 * h + q]);
+            }
           }
         }
         if constexpr (HYD) {

@@ -51,7 +51,7 @@ def test_issued_flops_counts_tiles():
     # dense: every candidate listed, no pooled tiles; causal row I lists I + 1 blocks
     rp_dense = np.concatenate([[0], np.cumsum(np.arange(1, 5))])
     assert bench.issued_flops(rp_dense, 1, 1, 4, 64, True, dense=True) == \
-        (1 + 1 + 2 + 2) * (2.0 * 128 * 64 * 64 + 2.0 * 128 * 64 * 128)
+        (1 + 1 + 2 + 2) * (2.0 * 128 * 64 * 64 + 2.0 * 64 * 64 * 128)
 
 
 def test_dense_flops_formula():
