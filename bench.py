@@ -453,7 +453,7 @@ def gpu_arm(args):
                      "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": round(achieved / tc_peak, 4),
                      # the capture is of psa_attn at the workload's own routing
-                     "traffic": None if st.dense or st.hyd or args.density is not None else recorded_traffic(st.name),
+                     "traffic": None if st.dense or st.hyd else recorded_traffic(st.name, args.density),
                      "peak_source": peaks["source"] + " bf16 burst"},
         "kernels": {"pool_ms": None if st.dense else round(pool_avg, 4),
                     "hyd_stat_ms": round(stat_avg, 4) if st.hyd else None,
@@ -578,11 +578,12 @@ def bwd_arm(args):
         dist.destroy_process_group()
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, density=None):
     """DRAM bytes per attention launch of this workload from the ncu record
     ``profiles/traffic.json`` (dram__bytes_read.sum + dram__bytes_write.sum of
     one captured launch), if the kernel source still hashes to the captured
-    one (else None: the counters no longer describe the kernel)."""
+    one and the capture used the same routing density override (else None:
+    the counters no longer describe the kernel or the run)."""
     import hashlib
 
     rec = os.path.join(ROOT, "profiles", "traffic.json")
@@ -593,7 +594,7 @@ def recorded_traffic(workload: str):
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     except (OSError, KeyError, ValueError):
         return None
-    if entry.get("attn_cu_sha256_prefix") != sha:
+    if entry.get("attn_cu_sha256_prefix") != sha or entry.get("density") != density:
         return None
     return int(entry["dram_bytes_per_launch"])
 

@@ -93,3 +93,14 @@ def test_reference_arm_prints_its_line_on_the_host():
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"]
+
+
+def test_recorded_traffic_matches_workload_and_density():
+    # the ncu record is used only for the workload, routing override and kernel
+    # source it was captured with
+    assert bench.recorded_traffic("no_such_workload") is None
+    assert bench.recorded_traffic("sweep_n64k", None) is None      # captured with --density 0.15
+    assert bench.recorded_traffic("dit_video_n32k", 0.5) is None    # captured with its own routing
+    for name, dens in (("dit_video_n32k", None), ("sweep_n64k", 0.15)):
+        v = bench.recorded_traffic(name, dens)
+        assert v is None or v > 0
