@@ -24,8 +24,9 @@
 // (tcgen05, TMEM accumulators, TMA operands) with one layout: warps 0-7 read
 // and write TMEM rows and do the elementwise work (warps w and w + 4 share
 // lane quarter w % 4, each taking half of a row's 64 columns), warp 8 loads
-// by TMA, warp 9 issues the MMAs and owns TMEM.  Every product keeps M = 128
-// rows:
+// by TMA, warp 9 issues the MMAs and owns TMEM (in the dq and dk, dv kernels
+// warp 9 issues the score products and warp 10 the accumulations).  Every
+// product keeps M = 128 rows:
 //   pseudo: S^T = Kbar_t Q_I^T, dP^T = Vsum_t dO_I^T   [128 pooled keys x 64 q]
 //           dVsum_t += Pi^T dO_I, dKbar_t += dA^T Q_I   [128 x d]
 //   dq:     S^T = K_t Q_I^T, dP^T = V_t dO_I^T           [128 keys x 64 q]
@@ -43,6 +44,10 @@ namespace {
 
 constexpr int kBwdThreads = 320;  // warps 0-7 elementwise, 8 TMA, 9 MMA + TMEM
 constexpr int kWarpTma = 8, kWarpMma = 9;
+// dq and dk, dv: a second MMA-issuing warp (10) for the accumulations, so
+// the scores of the next step and the accumulations of the current one issue
+// from two threads (an issue waits for the tensor core to accept it)
+constexpr int kKvThreads = 352, kWarpAcc = 10;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdArgs {
@@ -441,7 +446,7 @@ __device__ __forceinline__ DqUnit dq_unit(int u, const BwdArgs& g) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kKvThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVs,
@@ -464,8 +469,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* ds_free = bars + 20;   // its MMA is done
   uint64_t* dq_full = bars + 21;   // [2] a unit's dq^T is complete
   uint64_t* dq_empty = bars + 23;  // [2] read by the 8 elementwise warps
-  uint64_t* drain = bars + 25;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
+  uint64_t* drain = bars + 25;     // [2] teardown of the two issuers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -488,7 +493,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(u_free, 1);
     mbar_init(ds_full, 8);
     mbar_init(ds_free, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -572,98 +578,76 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     __syncwarp();
   } else if (warp == kWarpMma) {
-    // ---------------------------------------------------------- MMA issuer
+    // ---------------------------------------------------------- scores issuer
+    // S^T = K_t Q^T and dP^T = V_t dO^T of every step, in order
     if (lane == 0) {
       const uint64_t dQ = sdesc_sw128(smem_u32(smem), 16, 1024);
       const uint64_t dO = sdesc_sw128(smem_u32(smem + C::kQ), 16, 1024);
       const uint64_t dK = sdesc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(smem + C::kOffV), 16, 1024);
+      constexpr uint64_t kT16 = C::kTile >> 4;
+      int si = 0, ul = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++ul) {
+        const DqUnit x = dq_unit(u, g);
+        const int ub = ul & 1;
+        if (!(ok = mbar_wait(&u_full[ub], (ul >> 1) & 1, abort_flag, g.status))) break;
+        for (int t = 0; t < x.ntiles; ++t, ++si) {
+          const int ks = si % 3, vs = si & 1, b = si & 1;
+          if (!(ok = mbar_wait(&k_full[ks], (si / 3) & 1, abort_flag, g.status))) break;
+          if (!(ok = mbar_wait(&v_full[vs], (si >> 1) & 1, abort_flag, g.status))) break;
+          if (si >= 2 && !(ok = mbar_wait(&s_empty[b], ((si >> 1) - 1) & 1, abort_flag, g.status))) break;
+          tc_fence_after();
+          const uint64_t kt = dK + ks * kT16, vt = dV + vs * kT16;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ka = (kk >> 2) * 1024 + (kk & 3) * 2, kb = (kk >> 2) * 512 + (kk & 3) * 2;
+            tc_mma_bf16(tbase + 128 * b, kt + ka, dQ + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+            tc_mma_bf16(tbase + 128 * b + 64, vt + ka, dO + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[b]);
+          tc_commit(&v_free[vs]);
+          if (t == x.ntiles - 1) tc_commit(u_free);
+        }
+      }
+      tc_commit(&drain[0]);
+      drain_wait(&drain[0], 0);
+    }
+    __syncwarp();
+  } else if (warp == kWarpAcc) {
+    // ---------------------------------------------------------- dq issuer
+    // dq^T += K_t^T dS^T of every step, in order, once its dS^T is written (a
+    // unit's first step also once the epilogue of the unit two before has read
+    // the dq^T buffer it overwrites); each frees the dS^T tile and the key slot
+    if (lane == 0) {
       // key rows as the MN-major A of dq^T: M = features (64-feature atoms 16 KB apart)
       const uint64_t dKmn = sdesc_sw128(smem_u32(smem + C::kOffK), D == 128 ? 16384 : 0, 1024);
       const uint64_t dDs = sdesc_sw128(smem_u32(sDs), 16, 1024);
       constexpr uint64_t kT16 = C::kTile >> 4;
-      // the steps whose dq MMA is pending (at most two: one S^T buffer each)
-      struct Pending {
-        int ul, first, last;  // the step's unit (by CTA-local index), first / last step of it
-      } pend[2];
-      int ul_s = 0, t_s = 0, si_s = 0, si_a = 0;
-      int u_s = blockIdx.x;
-      DqUnit xs;
-      if (u_s < units) xs = dq_unit(u_s, g);
+      int si = 0, ul = 0;
       bool ok = true;
-      long long idle_since = clock64();
-      while (ok && (u_s < units || si_a < si_s)) {
-        bool progress = false;
-        // scores of the next step
-        if (u_s < units && si_s - si_a < 2) {
-          const int ub = ul_s & 1, ks = si_s % 3, vs = si_s & 1, b = si_s & 1;
-          if (mbar_try_wait(&u_full[ub], (ul_s >> 1) & 1) && mbar_try_wait(&k_full[ks], (si_s / 3) & 1) &&
-              mbar_try_wait(&v_full[vs], (si_s >> 1) & 1) &&
-              (si_s < 2 || mbar_try_wait(&s_empty[b], ((si_s >> 1) - 1) & 1))) {
-            tc_fence_after();
-            const uint64_t kt = dK + ks * kT16, vt = dV + vs * kT16;
+      for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++ul) {
+        const DqUnit x = dq_unit(u, g);
+        const int ub = ul & 1;
+        for (int t = 0; t < x.ntiles; ++t, ++si) {
+          if (!(ok = mbar_wait(ds_full, si & 1, abort_flag, g.status))) break;
+          if (t == 0 && ul >= 2 && !(ok = mbar_wait(&dq_empty[ub], ((ul >> 1) - 1) & 1, abort_flag, g.status))) break;
+          tc_fence_after();
+          const uint32_t t_dq = tbase + 256 + 64 * ub;
+          const uint64_t a = dKmn + (si % 3) * kT16;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t ka = (kk >> 2) * 1024 + (kk & 3) * 2, kb = (kk >> 2) * 512 + (kk & 3) * 2;
-              tc_mma_bf16(tbase + 128 * b, kt + ka, dQ + kb, C::kIdescS, kk > 0 ? 1u : 0u);
-              tc_mma_bf16(tbase + 128 * b + 64, vt + ka, dO + kb, C::kIdescS, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(&s_full[b]);
-            tc_commit(&v_free[vs]);
-            const bool last = t_s == xs.ntiles - 1;
-            if (last) tc_commit(u_free);
-            pend[si_s & 1] = {ul_s, t_s == 0, last};
-            ++si_s;
-            if (last) {
-              ++ul_s;
-              t_s = 0;
-              u_s += gridDim.x;
-              if (u_s < units) xs = dq_unit(u_s, g);
-            } else {
-              ++t_s;
-            }
-            progress = true;
-          }
-        }
-        // dq of the oldest pending step
-        if (si_a < si_s) {
-          const Pending pa = pend[si_a & 1];
-          const int ub = pa.ul & 1;
-          if (mbar_try_wait(ds_full, si_a & 1)) {
-            // the unit's first dq MMA overwrites dq^T[ub]: the epilogue of the unit
-            // two before (same buffer) must have read it
-            const bool free_buf =
-                !pa.first || pa.ul < 2 || mbar_try_wait(&dq_empty[ub], ((pa.ul >> 1) - 1) & 1);
-            if (free_buf) {
-              tc_fence_after();
-              const uint32_t t_dq = tbase + 256 + 64 * ub;
-              const uint64_t a = dKmn + (si_a % 3) * kT16;
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk)  // K = 128 key rows
-                tc_mma_bf16(t_dq, a + 128 * kk, dDs + 128 * kk, C::kIdescAcc, (!pa.first || kk > 0) ? 1u : 0u);
-              tc_commit(ds_free);
-              tc_commit(&k_free[si_a % 3]);
-              if (pa.last) tc_commit(&dq_full[ub]);
-              ++si_a;
-              progress = true;
-            }
-          }
-        }
-        if (progress) {
-          idle_since = clock64();
-        } else if (*abort_flag) {
-          ok = false;
-        } else if (clock64() - idle_since > kWaitCycles) {
-          *abort_flag = 1;
-          record_status(g.status, kStatusTimeout);
-          ok = false;
+          for (int kk = 0; kk < 8; ++kk)  // K = 128 key rows
+            tc_mma_bf16(t_dq, a + 128 * kk, dDs + 128 * kk, C::kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(ds_free);
+          tc_commit(&k_free[si % 3]);
+          if (t == x.ntiles - 1) tc_commit(&dq_full[ub]);
         }
       }
-      tc_commit(drain);
-      drain_wait(drain, 0);
+      tc_commit(&drain[1]);
+      drain_wait(&drain[1], 0);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ elementwise
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + lane;  // TMEM lane: key row of S^T, feature row of dq^T
@@ -786,7 +770,7 @@ struct KvMeta {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kKvThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const BwdArgs g, const float* __restrict__ dkbar, const float* __restrict__ dvsum,
@@ -809,8 +793,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* pd_free = bars + 11;
   uint64_t* acc_full = bars + 12;   // dK^T, dV^T of the item complete
   uint64_t* acc_empty = bars + 13;  // read by the 4 warps
-  uint64_t* drain = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* drain = bars + 14;     // [2] teardown of the two issuers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -828,7 +812,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(pd_free, 1);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -951,101 +936,93 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     __syncwarp();
   } else if (warp == kWarpMma) {
-    // ---------------------------------------------------------- MMA issuer
+    // ---------------------------------------------------------- scores issuer
+    // S = Q_p K_J^T and dP = dO_p V_J^T of every step, in order: a step's
+    // rows landed and its S / dP buffer read by the elementwise warps.
     if (lane == 0) {
       const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t dSt = sdesc_sw128(smem_u32(stage(0)), 16, 1024);
-      // q / dO pair rows as the MN-major A of dK^T / dV^T: M = features (atoms 16 KB apart)
+      constexpr uint64_t kSt16 = C::kStage >> 4, kPair16 = C::kPair >> 4;
+      int sc = 0, il = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++il) {
+        if (!(ok = mbar_wait(item_full, il & 1, abort_flag, g.status))) break;
+        for (;;) {
+          const int s = sc & 1, b = sc & 1;
+          if (!(ok = mbar_wait(&full[s], (sc >> 1) & 1, abort_flag, g.status))) break;
+          if (sc >= 2 && !(ok = mbar_wait(&s_empty[b], ((sc >> 1) - 1) & 1, abort_flag, g.status))) break;
+          volatile KvMeta* m = meta(s);
+          const bool has = m->Ia >= 0;
+          const bool last = m->last != 0;
+          tc_fence_after();
+          if (has) {
+            const uint64_t q = dSt + s * kSt16, o = q + kPair16;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t ka = (kk >> 2) * 1024 + (kk & 3) * 2, kb = (kk >> 2) * 512 + (kk & 3) * 2;
+              tc_mma_bf16(tbase + 128 * b, q + ka, dK + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+              tc_mma_bf16(tbase + 128 * b + 64, o + ka, dV + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(&s_full[b]);
+          ++sc;
+          if (last) break;
+        }
+      }
+      tc_commit(&drain[0]);
+      drain_wait(&drain[0], 0);
+    }
+    __syncwarp();
+  } else if (warp == kWarpAcc) {
+    // ---------------------------------------------------------- accumulation issuer
+    // dV^T += dO_p^T P and dK^T += Q_p^T dS of every step, in order, once its P
+    // and dS are written (and, for an item's first step, once the epilogue has
+    // read the previous item's accumulators); each frees the step's stage and
+    // the P / dS tiles, and the item's last frees K_J, V_J and completes the item.
+    if (lane == 0) {
       const uint64_t dStMN = sdesc_sw128(smem_u32(stage(0)), D == 128 ? 16384 : 0, 1024);
       const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
       const uint64_t dDs = sdesc_sw128(smem_u32(sDs), 16, 1024);
       constexpr uint64_t kSt16 = C::kStage >> 4, kPair16 = C::kPair >> 4;
-      // Issue whichever is ready: the scores of the next step (an S / dP
-      // buffer free, its rows landed) or the accumulation of the oldest
-      // pending step (its P and dS written), so a step's stage is released as
-      // early as its accumulation can run.
-      struct Pending {
-        int il, first, last, has;  // item (CTA-local index), first / last step of it, any rows
-      } pend[2];
-      int sc_s = 0, sc_a = 0, il_s = 0;
-      int it_s = blockIdx.x;
-      bool first_step = true;   // the next S step opens its item
-      bool acc_started = false; // an accumulation of the current item has run
+      int sc = 0, il = 0;
       bool ok = true;
-      long long idle_since = clock64();
-      while (ok && (it_s < items || sc_a < sc_s)) {
-        bool progress = false;
-        if (it_s < items && sc_s - sc_a < 2) {
-          const int s = sc_s & 1, b = sc_s & 1;
-          if (mbar_try_wait(item_full, il_s & 1) && mbar_try_wait(&full[s], (sc_s >> 1) & 1) &&
-              (sc_s < 2 || mbar_try_wait(&s_empty[b], ((sc_s >> 1) - 1) & 1))) {
-            volatile KvMeta* m = meta(s);
-            const bool has = m->Ia >= 0;
-            const bool last = m->last != 0;
-            tc_fence_after();
-            if (has) {
-              const uint64_t q = dSt + s * kSt16, o = q + kPair16;
+      for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++il) {
+        bool first = true, acc_started = false;
+        for (;;) {
+          const int ss = sc & 1;
+          if (!(ok = mbar_wait(pd_full, sc & 1, abort_flag, g.status))) break;
+          volatile KvMeta* m = meta(ss);
+          const bool has = m->Ia >= 0;
+          const bool last = m->last != 0;
+          if (first && il >= 1 && !(ok = mbar_wait(acc_empty, (il - 1) & 1, abort_flag, g.status))) break;
+          tc_fence_after();
+          if (has) {
+            const uint64_t q = dStMN + ss * kSt16, o = q + kPair16;
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t ka = (kk >> 2) * 1024 + (kk & 3) * 2, kb = (kk >> 2) * 512 + (kk & 3) * 2;
-                tc_mma_bf16(tbase + 128 * b, q + ka, dK + kb, C::kIdescS, kk > 0 ? 1u : 0u);
-                tc_mma_bf16(tbase + 128 * b + 64, o + ka, dV + kb, C::kIdescS, kk > 0 ? 1u : 0u);
-              }
+            for (int kk = 0; kk < 8; ++kk) {  // K = 128 query rows
+              const uint32_t acc = (acc_started || kk > 0) ? 1u : 0u;
+              tc_mma_bf16(t_dv, o + 128 * kk, dP + 128 * kk, C::kIdescAcc, acc);
+              tc_mma_bf16(t_dk, q + 128 * kk, dDs + 128 * kk, C::kIdescAcc, acc);
             }
-            tc_commit(&s_full[b]);
-            pend[sc_s & 1] = {il_s, first_step ? 1 : 0, last ? 1 : 0, has ? 1 : 0};
-            ++sc_s;
-            first_step = last;
-            if (last) {
-              ++il_s;
-              it_s += gridDim.x;
-            }
-            progress = true;
+            acc_started = true;
           }
-        }
-        if (sc_a < sc_s) {
-          const Pending pa = pend[sc_a & 1];
-          if (mbar_try_wait(pd_full, sc_a & 1) &&
-              (!pa.first || pa.il < 1 || mbar_try_wait(acc_empty, (pa.il - 1) & 1))) {
-            const int ss = sc_a & 1;
-            tc_fence_after();
-            if (pa.has) {
-              const uint64_t q = dStMN + ss * kSt16, o = q + kPair16;
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {  // K = 128 query rows
-                const uint32_t acc = (acc_started || kk > 0) ? 1u : 0u;
-                tc_mma_bf16(t_dv, o + 128 * kk, dP + 128 * kk, C::kIdescAcc, acc);
-                tc_mma_bf16(t_dk, q + 128 * kk, dDs + 128 * kk, C::kIdescAcc, acc);
-              }
-              acc_started = true;
-            }
-            tc_commit(pd_free);
-            tc_commit(&stage_free[ss]);
-            if (pa.last) {
-              tc_commit(acc_full);
-              tc_commit(item_free);
-              acc_started = false;
-            }
-            ++sc_a;
-            progress = true;
+          tc_commit(pd_free);
+          tc_commit(&stage_free[ss]);
+          if (last) {
+            tc_commit(acc_full);
+            tc_commit(item_free);
           }
-        }
-        if (progress) {
-          idle_since = clock64();
-        } else if (*abort_flag) {
-          ok = false;
-        } else if (clock64() - idle_since > kWaitCycles) {
-          *abort_flag = 1;
-          record_status(g.status, kStatusTimeout);
-          ok = false;
+          first = false;
+          ++sc;
+          if (last) break;
         }
       }
-      tc_commit(drain);
-      drain_wait(drain, 0);
+      tc_commit(&drain[1]);
+      drain_wait(&drain[1], 0);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
     // ---------------------------------------------------------- elementwise
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + lane;  // TMEM lane: query row of the pair (S, dP); feature row (dK^T, dV^T)
@@ -1209,7 +1186,7 @@ cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t st) {
   {
     if ((e = set_smem(bwd_dq_kernel<D>, DqCfg<D>::kSmem)) != cudaSuccess) return e;
     const int units = BH * M;
-    bwd_dq_kernel<D><<<units < sms ? units : sms, kBwdThreads, DqCfg<D>::kSmem, st>>>(
+    bwd_dq_kernel<D><<<units < sms ? units : sms, kKvThreads, DqCfg<D>::kSmem, st>>>(
         mq, mdo, mk, mv, mkb, mvs, g, reinterpret_cast<__nv_bfloat16*>(a.dq));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -1217,7 +1194,7 @@ cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t st) {
   {
     if ((e = set_smem(bwd_dkdv_kernel<D>, KvCfg<D>::kSmem)) != cudaSuccess) return e;
     const int items = BH * M;
-    bwd_dkdv_kernel<D><<<items < sms ? items : sms, kBwdThreads, KvCfg<D>::kSmem, st>>>(
+    bwd_dkdv_kernel<D><<<items < sms ? items : sms, kKvThreads, KvCfg<D>::kSmem, st>>>(
         mq, mdo, mk, mv, g, a.dkbar, a.dvsum, reinterpret_cast<__nv_bfloat16*>(a.dk),
         reinterpret_cast<__nv_bfloat16*>(a.dv));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
