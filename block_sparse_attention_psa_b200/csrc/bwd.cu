@@ -42,12 +42,12 @@
 namespace psa {
 namespace {
 
-constexpr int kBwdThreads = 320;  // warps 0-7 elementwise, 8 TMA, 9 MMA + TMEM
-constexpr int kWarpTma = 8, kWarpMma = 9;
-// dq and dk, dv: a second MMA-issuing warp (10) for the accumulations, so
-// the scores of the next step and the accumulations of the current one issue
-// from two threads (an issue waits for the tensor core to accept it)
-constexpr int kKvThreads = 352, kWarpAcc = 10;
+// Warps 0-7 elementwise, 8 TMA, 9 the score products (and TMEM), 10 the
+// accumulations: the scores of the next step and the accumulations of the
+// current one issue from two threads (an issue waits for the tensor core to
+// accept it).
+constexpr int kBwdThreads = 352;
+constexpr int kWarpTma = 8, kWarpMma = 9, kWarpAcc = 10;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdArgs {
@@ -186,8 +186,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* s_empty = bars + 7;     // [2] read by the 4 elementwise warps
   uint64_t* pd_full = bars + 9;     // Pi^T, dA^T written (4 warps)
   uint64_t* pd_free = bars + 10;    // their MMAs are done
-  uint64_t* done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* done = bars + 11;       // every accumulation MMA is done
+  uint64_t* drain_s = bars + 12;    // teardown of the scores issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(pd_full, 8);
     mbar_init(pd_free, 1);
     mbar_init(done, 1);
+    mbar_init(drain_s, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -256,51 +258,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     __syncwarp();
   } else if (warp == kWarpMma) {
+    // ---------------------------------------------------------- scores issuer
     if (lane == 0) {
       bool ok = n == 0 || mbar_wait(kv_full, 0, abort_flag, g.status);
       const uint64_t dKb = sdesc_sw128(smem_u32(sKb), 16, 1024);
       const uint64_t dVs = sdesc_sw128(smem_u32(sVs), 16, 1024);
       const uint64_t dStage = sdesc_sw128(smem_u32(smem + C::kOffStage), 16, 1024);
-      // the same q / dO tiles as MN-major B operands: N = D (atoms of 64 features 8 KB apart)
+      constexpr uint64_t kSt16 = C::kStage >> 4, kQ16 = C::kQ >> 4;
+      for (int i = 0; ok && i < n; ++i) {
+        const int s = i & 1, b = i & 1;
+        if (!(ok = mbar_wait(&full[s], (i >> 1) & 1, abort_flag, g.status))) break;
+        if (i >= 2 && !(ok = mbar_wait(&s_empty[b], ((i >> 1) - 1) & 1, abort_flag, g.status))) break;
+        tc_fence_after();
+        const uint64_t q = dStage + s * kSt16, o = q + kQ16;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ka = (kk >> 2) * 1024 + (kk & 3) * 2, kb = (kk >> 2) * 512 + (kk & 3) * 2;
+          tc_mma_bf16(tbase + 128 * b, dKb + ka, q + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+          tc_mma_bf16(tbase + 128 * b + 64, dVs + ka, o + kb, C::kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[b]);
+      }
+      tc_commit(drain_s);
+      drain_wait(drain_s, 0);
+    }
+    __syncwarp();
+  } else if (warp == kWarpAcc) {
+    // ---------------------------------------------------------- accumulation issuer
+    // dVsum_t += Pi^T dO and dKbar_t += dA^T Q of every step once its Pi^T and
+    // dA^T are written; `done` completes after the last (the elementwise
+    // warps saw every step's scores complete before writing its Pi^T, dA^T)
+    if (lane == 0) {
+      // the q / dO tiles as MN-major B operands: N = D (atoms of 64 features 8 KB apart)
       const uint64_t dStageMN = sdesc_sw128(smem_u32(smem + C::kOffStage), 8192, 1024);
       const uint64_t dPi = sdesc_sw128(smem_u32(sPi), 16, 1024);
       const uint64_t dDa = sdesc_sw128(smem_u32(sDa), 16, 1024);
       constexpr uint64_t kSt16 = C::kStage >> 4, kQ16 = C::kQ >> 4;
-      for (int i = 0; ok && i <= n; ++i) {
-        if (i < n) {
-          const int s = i & 1, b = i & 1;
-          if (!(ok = mbar_wait(&full[s], (i >> 1) & 1, abort_flag, g.status))) break;
-          if (i >= 2 && !(ok = mbar_wait(&s_empty[b], ((i >> 1) - 1) & 1, abort_flag, g.status))) break;
-          tc_fence_after();
-          const uint64_t q = dStage + s * kSt16, o = q + kQ16;
+      bool ok = true;
+      for (int j = 0; ok && j < n; ++j) {
+        const int sj = j & 1;
+        if (!(ok = mbar_wait(pd_full, j & 1, abort_flag, g.status))) break;
+        tc_fence_after();
+        const uint64_t q = dStageMN + sj * kSt16, o = q + kQ16;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ka = (kk >> 2) * 1024 + (kk & 3) * 2, kb = (kk >> 2) * 512 + (kk & 3) * 2;
-            tc_mma_bf16(tbase + 128 * b, dKb + ka, q + kb, C::kIdescS, kk > 0 ? 1u : 0u);
-            tc_mma_bf16(tbase + 128 * b + 64, dVs + ka, o + kb, C::kIdescS, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&s_full[b]);
+        for (int kk = 0; kk < 4; ++kk) {  // K = 64 queries
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+          tc_mma_bf16(t_acc_vs, dPi + kk * 2, o + 128 * kk, C::kIdescAcc, acc);
+          tc_mma_bf16(t_acc_kb, dDa + kk * 2, q + 128 * kk, C::kIdescAcc, acc);
         }
-        if (i >= 1) {
-          const int j = i - 1, sj = j & 1;
-          if (!(ok = mbar_wait(pd_full, j & 1, abort_flag, g.status))) break;
-          tc_fence_after();
-          const uint64_t q = dStageMN + sj * kSt16, o = q + kQ16;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {  // K = 64 queries
-            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-            tc_mma_bf16(t_acc_vs, dPi + kk * 2, o + 128 * kk, C::kIdescAcc, acc);
-            tc_mma_bf16(t_acc_kb, dDa + kk * 2, q + 128 * kk, C::kIdescAcc, acc);
-          }
-          tc_commit(pd_free);
-          tc_commit(&stage_free[sj]);
-        }
+        tc_commit(pd_free);
+        tc_commit(&stage_free[sj]);
       }
       tc_commit(done);
       drain_wait(done, 0);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ elementwise
     const int quarter = warp & 3, half = warp >> 2;
     const int j = quarter * 32 + lane;       // TMEM lane = pooled key of the tile
@@ -446,7 +459,7 @@ __device__ __forceinline__ DqUnit dq_unit(int u, const BwdArgs& g) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kKvThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVs,
@@ -770,7 +783,7 @@ struct KvMeta {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kKvThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const BwdArgs g, const float* __restrict__ dkbar, const float* __restrict__ dvsum,
@@ -1186,7 +1199,7 @@ cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t st) {
   {
     if ((e = set_smem(bwd_dq_kernel<D>, DqCfg<D>::kSmem)) != cudaSuccess) return e;
     const int units = BH * M;
-    bwd_dq_kernel<D><<<units < sms ? units : sms, kKvThreads, DqCfg<D>::kSmem, st>>>(
+    bwd_dq_kernel<D><<<units < sms ? units : sms, kBwdThreads, DqCfg<D>::kSmem, st>>>(
         mq, mdo, mk, mv, mkb, mvs, g, reinterpret_cast<__nv_bfloat16*>(a.dq));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -1194,7 +1207,7 @@ cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t st) {
   {
     if ((e = set_smem(bwd_dkdv_kernel<D>, KvCfg<D>::kSmem)) != cudaSuccess) return e;
     const int items = BH * M;
-    bwd_dkdv_kernel<D><<<items < sms ? items : sms, kKvThreads, KvCfg<D>::kSmem, st>>>(
+    bwd_dkdv_kernel<D><<<items < sms ? items : sms, kBwdThreads, KvCfg<D>::kSmem, st>>>(
         mq, mdo, mk, mv, g, a.dkbar, a.dvsum, reinterpret_cast<__nv_bfloat16*>(a.dk),
         reinterpret_cast<__nv_bfloat16*>(a.dv));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
