@@ -402,6 +402,7 @@ int psa_attn_bwd(const psa_bf16_t* q, const psa_bf16_t* k, const psa_bf16_t* v, 
   a.d = d;
   a.causal = causal;
   a.status = reinterpret_cast<int*>(ws);
+  a.sched = reinterpret_cast<int*>(ws) + 8;
   // scratch of the backward: regions the forward calls use only within a call
   a.bits = reinterpret_cast<uint32_t*>(ws + L.row_bits);
   a.nlse2 = reinterpret_cast<float*>(ws + L.row_lse2);

@@ -61,6 +61,7 @@ struct BwdArgs {
   float sl;               // log2(e) / sqrt(d)
   float tau;              // 1 / sqrt(d)
   int* status;
+  int* sched;             // ticket counter of the dk, dv item scheduler (zero at the call's start)
 };
 
 // 32 bf16 (columns 32*half ..) of row r of a 128-byte-swizzled tile (row r,
@@ -809,10 +810,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* drain = bars + 14;     // [2] teardown of the two issuers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* iring = reinterpret_cast<volatile int*>(bars + 17);  // [4] item ids in flight
+  uint64_t* id_full = bars + 19;    // [4] an item id published (producer)
+  uint64_t* id_empty = bars + 23;   // [4] read by its 10 consumers (both issuers, 8 elementwise warps)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int items = g.BH * g.M;
+  // Dynamic item scheduler: a CTA's first item is blockIdx.x, each later one
+  // the next ticket of the call's counter (after the grid's first items), so
+  // CTAs that drew key blocks listed by few query blocks take more of them.
+  // The producer draws and publishes the CTA's il-th item in slot il % 4;
+  // every other role reads the slots in order; -1 ends the sequence.
+  auto publish = [&](int il) -> int {
+    int it;
+    if (il == 0) {
+      it = static_cast<int>(blockIdx.x) < items ? static_cast<int>(blockIdx.x) : -1;
+    } else {
+      it = static_cast<int>(gridDim.x) + atomicAdd(g.sched, 1);
+      if (it >= items) it = -1;
+    }
+    const int slot = il & 3;
+    if (il >= 4 && !mbar_wait(&id_empty[slot], ((il >> 2) - 1) & 1, abort_flag, g.status)) return -1;
+    iring[slot] = it;
+    mbar_arrive(&id_full[slot]);
+    return it;
+  };
+  auto fetch = [&](int il) -> int {  // by lane 0 of a consuming warp
+    const int slot = il & 3;
+    if (!mbar_wait(&id_full[slot], (il >> 2) & 1, abort_flag, g.status)) return -1;
+    const int it = iring[slot];
+    mbar_arrive(&id_empty[slot]);
+    return it;
+  };
   if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&id_full[i], 1);
+      mbar_init(&id_empty[i], 10);
+    }
     mbar_init(item_full, 1);
     mbar_init(item_free, 1);
     for (int i = 0; i < 2; ++i) {
@@ -845,10 +879,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == kWarpTma) {
     // ---------------------------------------------------------- producer
     // the query blocks that list key block J, in pairs
-    int sc = 0, il = 0;
+    int sc = 0;
     int st_issued[2] = {0, 0}, it_issued = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++il) {
+    for (int il = 0; ok; ++il) {
+      int it = -1;
+      if (lane == 0) it = publish(il);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      if (it < 0) break;
       const int bh = it / g.M, J = it - bh * g.M;
       if (lane == 0) {
         if (il >= 1) ok = mbar_wait(item_free, (il - 1) & 1, abort_flag, g.status);
@@ -957,9 +995,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dV = sdesc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t dSt = sdesc_sw128(smem_u32(stage(0)), 16, 1024);
       constexpr uint64_t kSt16 = C::kStage >> 4, kPair16 = C::kPair >> 4;
-      int sc = 0, il = 0;
+      int sc = 0;
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++il) {
+      for (int il = 0; ok; ++il) {
+        if (fetch(il) < 0) break;
         if (!(ok = mbar_wait(item_full, il & 1, abort_flag, g.status))) break;
         for (;;) {
           const int s = sc & 1, b = sc & 1;
@@ -998,9 +1037,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
       const uint64_t dDs = sdesc_sw128(smem_u32(sDs), 16, 1024);
       constexpr uint64_t kSt16 = C::kStage >> 4, kPair16 = C::kPair >> 4;
-      int sc = 0, il = 0;
+      int sc = 0;
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++il) {
+      for (int il = 0; ok; ++il) {
+        if (fetch(il) < 0) break;
         bool first = true, acc_started = false;
         for (;;) {
           const int ss = sc & 1;
@@ -1041,9 +1081,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int r = quarter * 32 + lane;  // TMEM lane: query row of the pair (S, dP); feature row (dK^T, dV^T)
     const int c0 = 32 * half;           // this thread's 32 key columns
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    int sc = 0, il = 0;
+    int sc = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++il) {
+    for (int il = 0; ok; ++il) {
+      int it = -1;
+      if (lane == 0) it = fetch(il);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      if (it < 0) break;
       const int bh = it / g.M, J = it - bh * g.M;
       bool any = false;
       for (;;) {
@@ -1163,6 +1207,7 @@ cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t st) {
   g.sl = kLog2e / sqrtf(static_cast<float>(D));
   g.tau = 1.0f / sqrtf(static_cast<float>(D));
   g.status = a.status;
+  g.sched = a.sched;
   const int sms = device_sm_count();
   cudaError_t e;
   // delta and -lse log2 e

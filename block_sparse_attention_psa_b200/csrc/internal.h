@@ -143,6 +143,7 @@ struct BwdLaunch {
   uint16_t* dv;
   int BH, N, M, d, causal;
   int* status;
+  int* sched;            // ticket counter of the dk, dv item scheduler (zeroed header word)
   // workspace
   uint32_t* bits;        // [BH*M][ceil(M/32)]
   float* nlse2;          // [BH*N]
