@@ -426,7 +426,7 @@ struct DqCfg {
   static constexpr int kOffDs = kOffV + kVSlots * kTile;
   static constexpr int kOffNl = kOffDs + 128 * 128;         // [2][-lse log2e 64, D 64]
   static constexpr int kOffBars = kOffNl + 2 * 512;
-  static constexpr int kSmem = kOffBars + 256 + 1024;
+  static constexpr int kSmem = kOffBars + 512 + 1024;  // 512 B: barriers, TMEM slot, unit ring
   static_assert(kSmem <= 232448, "shared memory of one CTA");
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);
   // dq^T [D x 64 q] += K^T (A: M = features, MN-major) . dS^T (B: N = q, MN-major)
@@ -486,10 +486,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* drain = bars + 25;     // [2] teardown of the two issuers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* uring = reinterpret_cast<volatile int*>(bars + 28);  // [4] unit ids in flight
+  uint64_t* id_full = bars + 30;   // [4] a unit id published (producer)
+  uint64_t* id_empty = bars + 34;  // [4] read by its 10 consumers (both issuers, 8 elementwise warps)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int units = g.BH * g.M;
+  // Dynamic unit scheduler, as in the forward: a CTA's first unit comes from
+  // blockIdx.x, each later one from the next ticket of the call's counter;
+  // ticket t is query block M - 1 - t % M of head t / M (largest first, so
+  // long causal units start early).  The producer publishes the CTA's ul-th
+  // unit in slot ul % 4; the other roles read the slots in order; -1 ends.
+  auto publish = [&](int ul) -> int {
+    int t;
+    if (ul == 0) {
+      t = static_cast<int>(blockIdx.x) < units ? static_cast<int>(blockIdx.x) : -1;
+    } else {
+      t = static_cast<int>(gridDim.x) + atomicAdd(g.sched + 1, 1);
+      if (t >= units) t = -1;
+    }
+    const int u = t < 0 ? -1 : (t / g.M) * g.M + g.M - 1 - t % g.M;
+    const int slot = ul & 3;
+    if (ul >= 4 && !mbar_wait(&id_empty[slot], ((ul >> 2) - 1) & 1, abort_flag, g.status)) return -1;
+    uring[slot] = u;
+    mbar_arrive(&id_full[slot]);
+    return u;
+  };
+  auto fetch = [&](int ul) -> int {  // by lane 0 of a consuming warp
+    const int slot = ul & 3;
+    if (!mbar_wait(&id_full[slot], (ul >> 2) & 1, abort_flag, g.status)) return -1;
+    const int u = uring[slot];
+    mbar_arrive(&id_empty[slot]);
+    return u;
+  };
   if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&id_full[i], 1);
+      mbar_init(&id_empty[i], 10);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&u_full[i], 1);
       mbar_init(&nl_free[i], 8);
@@ -524,10 +558,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == kWarpTma) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
-      int si = 0, ul = 0;
+      int si = 0;
       int k_iss[3] = {0, 0, 0}, v_iss[2] = {0, 0}, u_iss[2] = {0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++ul) {
+      for (int ul = 0; ok; ++ul) {
+        const int u = publish(ul);
+        if (u < 0) break;
         const DqUnit x = dq_unit(u, g);
         const int ub = ul & 1;
         // q, dO stage: the previous unit's scores are done; its -lse / D slot: read
@@ -600,9 +636,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dK = sdesc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(smem + C::kOffV), 16, 1024);
       constexpr uint64_t kT16 = C::kTile >> 4;
-      int si = 0, ul = 0;
+      int si = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++ul) {
+      for (int ul = 0; ok; ++ul) {
+        const int u = fetch(ul);
+        if (u < 0) break;
         const DqUnit x = dq_unit(u, g);
         const int ub = ul & 1;
         if (!(ok = mbar_wait(&u_full[ub], (ul >> 1) & 1, abort_flag, g.status))) break;
@@ -638,9 +676,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dKmn = sdesc_sw128(smem_u32(smem + C::kOffK), D == 128 ? 16384 : 0, 1024);
       const uint64_t dDs = sdesc_sw128(smem_u32(sDs), 16, 1024);
       constexpr uint64_t kT16 = C::kTile >> 4;
-      int si = 0, ul = 0;
+      int si = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++ul) {
+      for (int ul = 0; ok; ++ul) {
+        const int u = fetch(ul);
+        if (u < 0) break;
         const DqUnit x = dq_unit(u, g);
         const int ub = ul & 1;
         for (int t = 0; t < x.ntiles; ++t, ++si) {
@@ -667,8 +707,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int r = quarter * 32 + lane;  // TMEM lane: key row of S^T, feature row of dq^T
     const int c0 = 32 * half;           // this thread's 32 query columns
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    int sc = 0, ul = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x, ++ul) {
+    int sc = 0;
+    for (int ul = 0;; ++ul) {
+      int u = -1;
+      if (lane == 0) u = fetch(ul);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (u < 0) break;
       const DqUnit x = dq_unit(u, g);
       const int ub = ul & 1;
       if (!mbar_wait(&u_full[ub], (ul >> 1) & 1, abort_flag, g.status)) break;
