@@ -12,7 +12,12 @@
  *    where a comment says "host".  The library never allocates device memory
  *    and never frees what it is given.
  *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
- *    NULL = the legacy default stream) and returns a status code.
+ *    NULL = the legacy default stream) and returns a status code.  The
+ *    forward path's kernels are programmatic dependent launches: each may
+ *    start its setup while the kernel before it on the stream drains, and
+ *    waits on the device before touching memory, so stream order holds for
+ *    every read and write; captured into a CUDA graph they become
+ *    programmatic edges.
  *  - Arguments are validated on the host before any launch: a bad argument
  *    returns an error code and launches nothing.  The tensors must live on
  *    the CURRENT device (cudaSetDevice): a call whose main input or output
