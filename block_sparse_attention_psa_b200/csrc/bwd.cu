@@ -24,9 +24,9 @@
 // (tcgen05, TMEM accumulators, TMA operands) with one layout: warps 0-7 read
 // and write TMEM rows and do the elementwise work (warps w and w + 4 share
 // lane quarter w % 4, each taking half of a row's 64 columns), warp 8 loads
-// by TMA, warp 9 issues the MMAs and owns TMEM (in the dq and dk, dv kernels
-// warp 9 issues the score products and warp 10 the accumulations).  Every
-// product keeps M = 128 rows:
+// by TMA, warp 9 issues the score products and owns TMEM, warp 10 issues the
+// accumulations; the dq and dk, dv kernels draw their units and items from
+// dynamic schedulers.  Every product keeps M = 128 rows:
 //   pseudo: S^T = Kbar_t Q_I^T, dP^T = Vsum_t dO_I^T   [128 pooled keys x 64 q]
 //           dVsum_t += Pi^T dO_I, dKbar_t += dA^T Q_I   [128 x d]
 //   dq:     S^T = K_t Q_I^T, dP^T = V_t dO_I^T           [128 keys x 64 q]
