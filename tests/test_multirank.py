@@ -41,11 +41,13 @@ def _worker(rank, world, port, out):
 def test_two_ranks_max_timing_and_distinct_problems():
     world = 2
     port = _free_port()
-    manager = mp.Manager()
-    out = manager.dict()
-    mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+    # the manager's server process is started by spawn too: nothing here forks
+    with mp.get_context("spawn").Manager() as manager:
+        out = manager.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = {rank: out[rank] for rank in range(world)}
     for rank in range(world):
-        total, digests = out[rank]
+        total, digests = res[rank]
         assert total == 15.0
         assert digests[0] != digests[1]          # independent seeded problems
 
